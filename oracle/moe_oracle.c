@@ -1,0 +1,363 @@
+/*
+ * moe_oracle.c -- plain, slow CPU oracle for the routed-experts MoE forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference leg of bench.py may load this library.  It shares
+ * no code, header, table or helper with the CUDA library under
+ * mixture_experts_routed_expert_b200/, and the CUDA library never calls it.
+ *
+ * Arithmetic: every dot product and every sum is accumulated in fp64 in
+ * ascending index order, on the exact values of the bf16 / E4M3 operands
+ * (E4M3 operands dequantised with their fp32 scales first).  Rounding to
+ * bf16 / E4M3 happens only where the method stores a value in that format.
+ *
+ * Sources (web pages, cited by title and section):
+ *  - "deepseek-ocr2-moe-experts" model card, description + "Usage":
+ *    out[t] = sum_k w[t,k] * down_e(SiLU(gate_e x_t) * up_e x_t), weight
+ *    layout gate_up_proj [E,2F,H], down_proj [E,H,F], top_k_index [T,K] int32,
+ *    top_k_weights [T,K] fp32; routing happens outside the op.
+ *  - "[Feature Request] - Supporting MegaKernel for DeepSeek Models",
+ *    "Layer Tensor Details": moe_topk_sigmoid_routing_layer (group-aware
+ *    sigmoid routing, num_groups=8, topk_group=4, routed_scaling_factor=2.5),
+ *    bf16_to_fp8_quantize (block 128, E4M3 + power-of-two scale),
+ *    moe_w13_fp8_layer / moe_w2_fp8_layer (per (row,128-col) fp32 weight
+ *    scales), moe_silu_mul_layer, moe_local_reduction (weighted sum over k).
+ *
+ * Parity pins: every exported function is pinned by tests under tests/
+ * (test_oracle_*.py) against library routines, closed forms, invariants and
+ * brute force; none is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Number formats                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Round v to the nearest number that has `p` significant bits and whose
+ * exponent is at least emin (below 2^emin the spacing stays 2^(emin-p+1),
+ * i.e. gradual underflow).  Ties go to the even neighbour: nearbyint() in the
+ * default rounding mode.  v/quantum is exact (power-of-two scaling). */
+static double round_sig(double v, int p, int emin) {
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e;
+    (void)frexp(fabs(v), &e);          /* |v| = m 2^e, m in [0.5,1) */
+    int lead = e - 1;                  /* exponent of the leading bit */
+    if (lead < emin) lead = emin;
+    double quantum = ldexp(1.0, lead - (p - 1));
+    return nearbyint(v / quantum) * quantum;
+}
+
+/* bf16: 8 significant bits, normal exponents from -126, largest finite
+ * (2 - 2^-7) 2^127.  Overflow after rounding gives infinity (IEEE RNE). */
+static double bf16_value(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+static uint16_t bf16_from_double(double v) {
+    if (isnan(v)) return 0x7FC0;
+    double r = round_sig(v, 8, -126);
+    const double maxf = ldexp(255.0, 120);         /* (2-2^-7) 2^127 */
+    if (fabs(r) > maxf) r = copysign(INFINITY, r);
+    float f = (float)r;                            /* exact */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+/* OCP 8-bit floating point, E4M3 ("fn" variant): 1 sign, 4 exponent bits
+ * (bias 7), 3 mantissa bits, no infinities, S.1111.111 = NaN, largest finite
+ * S.1111.110 = 448, smallest normal 2^-6, subnormal spacing 2^-9.
+ * The conversion is round-to-nearest-even with saturation of finite values
+ * to +-448. */
+static double e4m3_value(uint8_t c) {
+    int s = c >> 7, ex = (c >> 3) & 15, m = c & 7;
+    double mag;
+    if (ex == 15 && m == 7) return NAN;
+    if (ex == 0) mag = ldexp((double)m, -9);
+    else mag = ldexp(1.0 + m / 8.0, ex - 7);
+    return s ? -mag : mag;
+}
+
+static uint8_t e4m3_from_double(double v) {
+    if (isnan(v)) return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double r = fabs(round_sig(v, 4, -6));
+    if (r > 448.0) r = 448.0;                      /* satfinite */
+    if (r == 0.0) return sign;
+    if (r < ldexp(1.0, -6)) {                      /* subnormal: m * 2^-9 */
+        int m = (int)ldexp(r, 9);
+        return (uint8_t)(sign | m);
+    }
+    int e;
+    double fr = frexp(r, &e);                      /* r = fr 2^e */
+    int lead = e - 1;
+    int m = (int)((ldexp(fr, 1) - 1.0) * 8.0);     /* r/2^lead = 1 + m/8 */
+    return (uint8_t)(sign | ((lead + 7) << 3) | m);
+}
+
+/* Exported format helpers (pinned against torch's own conversions). */
+void oracle_bf16_from_f64(const double *v, int64_t n, uint16_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = bf16_from_double(v[i]);
+}
+void oracle_e4m3_from_f64(const double *v, int64_t n, uint8_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_from_double(v[i]);
+}
+void oracle_e4m3_to_f64(const uint8_t *c, int64_t n, double *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(c[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* S2: block-128 activation quantisation                                     */
+/* (MegaKernel DeepSeek layer table, bf16_to_fp8_quantize)                   */
+/* ------------------------------------------------------------------------ */
+
+/* Scale of one block: the smallest power of two s = 2^k with amax/s <= 448,
+ * with k clamped to [-127, 127] so that s is an unsigned-exponent (ue8m0)
+ * value; amax == 0 gives s = 1.  With amax = m 2^e, m in [0.5,1) and
+ * 448 = 0.875 2^9:  k = e - 9 when m <= 0.875, else e - 8. */
+static int block_scale_exp(double amax) {
+    if (amax == 0.0) return 0;
+    int e;
+    double m = frexp(amax, &e);
+    int k = (m <= 0.875) ? e - 9 : e - 8;
+    if (k < -127) k = -127;
+    if (k > 127) k = 127;
+    return k;
+}
+
+/* Quantise n_blocks consecutive blocks of 128 values (given as doubles that
+ * are exact bf16 values).  q = E4M3(v / s) elementwise, scale = s (fp32). */
+static void quantize_blocks(const double *v, int n_blocks, uint8_t *q, float *scale) {
+    for (int b = 0; b < n_blocks; ++b) {
+        const double *vb = v + (int64_t)b * 128;
+        double amax = 0.0;
+        for (int i = 0; i < 128; ++i) amax = fmax(amax, fabs(vb[i]));
+        int k = block_scale_exp(amax);
+        for (int i = 0; i < 128; ++i) q[(int64_t)b * 128 + i] = e4m3_from_double(ldexp(vb[i], -k));
+        scale[b] = (float)ldexp(1.0, k);
+    }
+}
+
+/* x: [rows, cols] bf16 bits, cols % 128 == 0 -> xq [rows, cols] E4M3 bits,
+ * scale [rows, cols/128] fp32. */
+void oracle_quantize_fp8_block128(const uint16_t *x, int64_t rows, int64_t cols,
+                                  uint8_t *xq, float *scale) {
+    int nb = (int)(cols / 128);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        double *tmp = (double *)malloc(sizeof(double) * cols);
+        for (int64_t c = 0; c < cols; ++c) tmp[c] = bf16_value(x[r * cols + c]);
+        quantize_blocks(tmp, nb, xq + r * cols, scale + r * nb);
+        free(tmp);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* S1: group-aware sigmoid top-k routing                                     */
+/* (MegaKernel DeepSeek layer table, moe_topk_sigmoid_routing_layer)         */
+/* ------------------------------------------------------------------------ */
+
+/* "a ranks before b": larger score first, lower index on equal scores. */
+static int ranks_before(float sa, int ia, float sb, int ib) {
+    return sa > sb || (sa == sb && ia < ib);
+}
+
+/* logits [T,E] fp32, bias [E] fp32.  Per token:
+ *   s_e = sigmoid(logit_e), computed in double and rounded to fp32;
+ *   c_e = s_e + bias_e (fp32 add);
+ *   group score = top1 + top2 of c inside each of num_groups equal groups
+ *                 (just top1 when a group holds one expert);
+ *   keep the topk_group best groups; choose the top_k best c among experts
+ *   of kept groups (ties: lower index);  w_k = (s_k / sum_j s_j) * scale,
+ *   sum_j in selection order, all fp32.
+ * Outputs top_k_index [T,K] int32 (selection order), top_k_weights [T,K]. */
+void oracle_route_sigmoid_grouped(const float *logits, const float *bias, int64_t T, int E,
+                                  int num_groups, int topk_group, int top_k, float scale,
+                                  int32_t *top_k_index, float *top_k_weights) {
+    int gsize = E / num_groups;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        float *s = (float *)malloc(sizeof(float) * E);
+        float *c = (float *)malloc(sizeof(float) * E);
+        float *gs = (float *)malloc(sizeof(float) * num_groups);
+        char *gkeep = (char *)calloc(num_groups, 1);
+        char *taken = (char *)calloc(E, 1);
+        for (int e = 0; e < E; ++e) {
+            double x = (double)logits[t * E + e];
+            s[e] = (float)(1.0 / (1.0 + exp(-x)));
+            c[e] = s[e] + bias[e];
+        }
+        for (int g = 0; g < num_groups; ++g) {
+            int b1 = -1, b2 = -1;
+            for (int e = g * gsize; e < (g + 1) * gsize; ++e) {
+                if (b1 < 0 || ranks_before(c[e], e, c[b1], b1)) { b2 = b1; b1 = e; }
+                else if (b2 < 0 || ranks_before(c[e], e, c[b2], b2)) { b2 = e; }
+            }
+            gs[g] = (b2 >= 0) ? c[b1] + c[b2] : c[b1];
+        }
+        for (int r = 0; r < topk_group; ++r) {
+            int best = -1;
+            for (int g = 0; g < num_groups; ++g)
+                if (!gkeep[g] && (best < 0 || ranks_before(gs[g], g, gs[best], best))) best = g;
+            gkeep[best] = 1;
+        }
+        for (int k = 0; k < top_k; ++k) {
+            int best = -1;
+            for (int e = 0; e < E; ++e)
+                if (gkeep[e / gsize] && !taken[e] && (best < 0 || ranks_before(c[e], e, c[best], best)))
+                    best = e;
+            taken[best] = 1;
+            top_k_index[t * top_k + k] = best;
+        }
+        float sum = 0.0f;
+        for (int k = 0; k < top_k; ++k) sum += s[top_k_index[t * top_k + k]];
+        for (int k = 0; k < top_k; ++k) {
+            float q = s[top_k_index[t * top_k + k]] / sum;
+            top_k_weights[t * top_k + k] = q * scale;
+        }
+        free(s); free(c); free(gs); free(gkeep); free(taken);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* S3: expert histogram, offsets and stable permutation                      */
+/* ------------------------------------------------------------------------ */
+
+/* idx [T*K] (slot = t*K + k).  counts[e] = slots routed to e;
+ * offsets = exclusive prefix of counts (E+1 entries);
+ * perm[p] = slot at permuted position p, positions grouped by expert and in
+ * ascending slot order inside an expert (p >= offsets[E] -> -1);
+ * inv[slot] = its position, -1 for expert ids outside [0,E). */
+void oracle_permute(const int32_t *idx, int64_t n_slots, int E, int32_t *counts,
+                    int32_t *offsets, int32_t *perm, int32_t *inv) {
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t i = 0; i < n_slots; ++i)
+        if (idx[i] >= 0 && idx[i] < E) counts[idx[i]]++;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *next = (int32_t *)malloc(sizeof(int32_t) * (E > 0 ? E : 1));
+    for (int e = 0; e < E; ++e) next[e] = offsets[e];
+    for (int64_t p = 0; p < n_slots; ++p) perm[p] = -1;
+    for (int64_t i = 0; i < n_slots; ++i) {
+        int e = idx[i];
+        if (e >= 0 && e < E) { perm[next[e]] = (int32_t)i; inv[i] = next[e]++; }
+        else inv[i] = -1;
+    }
+    free(next);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Routed-experts forward (S3..S6 / S7 collapsed into the definition)        */
+/* ------------------------------------------------------------------------ */
+
+static double silu(double g) { return g / (1.0 + exp(-g)); }
+
+/* bf16 weights.  x [T,H], gate_up [E,2F,H] (rows [0,F) gate, [F,2F) up),
+ * down [E,H,F], idx/w [T,K]; out [T,H] bf16.
+ * h is rounded to bf16 (the intermediate activation is stored in the
+ * activation dtype); y is not rounded; out = bf16(sum_k w y). */
+void oracle_moe_forward_bf16(const uint16_t *x, const uint16_t *gate_up, const uint16_t *down,
+                             const int32_t *idx, const float *w, int64_t T, int H, int F, int E,
+                             int K, uint16_t *out) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < T; ++t) {
+        double *xt = (double *)malloc(sizeof(double) * H);
+        double *acc = (double *)calloc(H, sizeof(double));
+        double *hb = (double *)malloc(sizeof(double) * F);
+        for (int i = 0; i < H; ++i) xt[i] = bf16_value(x[t * H + i]);
+        for (int k = 0; k < K; ++k) {
+            int e = idx[t * K + k];
+            if (e < 0 || e >= E) continue;
+            const uint16_t *G = gate_up + (int64_t)e * 2 * F * H;
+            const uint16_t *U = G + (int64_t)F * H;
+            const uint16_t *D = down + (int64_t)e * H * F;
+            for (int f = 0; f < F; ++f) {
+                double g = 0.0, u = 0.0;
+                for (int i = 0; i < H; ++i) {
+                    g += bf16_value(G[(int64_t)f * H + i]) * xt[i];
+                    u += bf16_value(U[(int64_t)f * H + i]) * xt[i];
+                }
+                hb[f] = bf16_value(bf16_from_double(silu(g) * u));
+            }
+            double wk = (double)w[t * K + k];
+            for (int j = 0; j < H; ++j) {
+                double y = 0.0;
+                for (int f = 0; f < F; ++f) y += bf16_value(D[(int64_t)j * F + f]) * hb[f];
+                acc[j] += wk * y;
+            }
+        }
+        for (int j = 0; j < H; ++j) out[t * H + j] = bf16_from_double(acc[j]);
+        free(xt); free(acc); free(hb);
+    }
+}
+
+/* FP8 E4M3 weights with fp32 scales per (row, 128-column block):
+ * w13 [E,2F,H] + w13_scale [E,2F,H/128], w2 [E,H,F] + w2_scale [E,H,F/128].
+ * x (bf16) is quantised per 128 columns by the S2 rule; h = bf16(SiLU(g) u)
+ * is quantised per 128 features by the same rule; every E4M3 operand is
+ * dequantised (code value * its block scale) before the fp64 dot products;
+ * out = bf16(sum_k w y). */
+void oracle_moe_forward_fp8(const uint16_t *x, const uint8_t *w13, const float *w13_scale,
+                            const uint8_t *w2, const float *w2_scale, const int32_t *idx,
+                            const float *w, int64_t T, int H, int F, int E, int K, uint16_t *out) {
+    int hb_n = H / 128, fb_n = F / 128;
+    double lut[256];                               /* value of every E4M3 code */
+    for (int c = 0; c < 256; ++c) lut[c] = e4m3_value((uint8_t)c);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < T; ++t) {
+        double *xt = (double *)malloc(sizeof(double) * H);
+        double *xd = (double *)malloc(sizeof(double) * H);
+        uint8_t *xq = (uint8_t *)malloc(H);
+        float *xs = (float *)malloc(sizeof(float) * hb_n);
+        double *acc = (double *)calloc(H, sizeof(double));
+        double *hv = (double *)malloc(sizeof(double) * F);
+        double *hd = (double *)malloc(sizeof(double) * F);
+        uint8_t *hq = (uint8_t *)malloc(F);
+        float *hs = (float *)malloc(sizeof(float) * fb_n);
+        for (int i = 0; i < H; ++i) xt[i] = bf16_value(x[t * H + i]);
+        quantize_blocks(xt, hb_n, xq, xs);
+        for (int i = 0; i < H; ++i) xd[i] = e4m3_value(xq[i]) * (double)xs[i / 128];
+        for (int k = 0; k < K; ++k) {
+            int e = idx[t * K + k];
+            if (e < 0 || e >= E) continue;
+            for (int f = 0; f < F; ++f) {
+                int64_t rg = (int64_t)e * 2 * F + f, ru = rg + F;
+                double g = 0.0, u = 0.0;
+                for (int i = 0; i < H; ++i) {
+                    g += lut[w13[rg * H + i]] * (double)w13_scale[rg * hb_n + i / 128] * xd[i];
+                    u += lut[w13[ru * H + i]] * (double)w13_scale[ru * hb_n + i / 128] * xd[i];
+                }
+                hv[f] = bf16_value(bf16_from_double(silu(g) * u));
+            }
+            quantize_blocks(hv, fb_n, hq, hs);
+            for (int f = 0; f < F; ++f) hd[f] = e4m3_value(hq[f]) * (double)hs[f / 128];
+            double wk = (double)w[t * K + k];
+            for (int j = 0; j < H; ++j) {
+                int64_t rd = (int64_t)e * H + j;
+                double y = 0.0;
+                for (int f = 0; f < F; ++f)
+                    y += lut[w2[rd * F + f]] * (double)w2_scale[rd * fb_n + f / 128] * hd[f];
+                acc[j] += wk * y;
+            }
+        }
+        for (int j = 0; j < H; ++j) out[t * H + j] = bf16_from_double(acc[j]);
+        free(xt); free(xd); free(xq); free(xs); free(acc); free(hv); free(hd); free(hq); free(hs);
+    }
+}
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
