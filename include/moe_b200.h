@@ -1,0 +1,190 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) routed-experts MoE library
+ * (libmoe_b200.so).
+ *
+ * The operation ("deepseek-ocr2-moe-experts" model card, description and
+ * "Usage"):
+ *
+ *     out[t] = sum_{k<K} w[t,k] * down_e( SiLU(gate_e x_t) * (up_e x_t) ),
+ *     e = top_k_index[t,k],
+ *
+ * with the argument order of the card's two ops
+ * (hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k).
+ * FP8 variants, the router and the quantiser follow the layer table of
+ * "[Feature Request] - Supporting MegaKernel for DeepSeek Models"
+ * ("Layer Tensor Details": moe_w13_fp8_layer, moe_silu_mul_layer,
+ * moe_w2_fp8_layer, moe_topk_sigmoid_routing_layer, bf16_to_fp8_quantize,
+ * moe_local_reduction).
+ *
+ * Conventions for every entry point:
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller; the
+ *    library allocates no device memory and keeps no per-call state.  Where
+ *    scratch memory is needed the caller passes a workspace of at least
+ *    moe_experts_workspace_size() bytes.
+ *  - Tensors are dense, row-major (last dimension contiguous), with the
+ *    layouts written beside each argument.  bf16 = IEEE bfloat16,
+ *    e4m3 = OCP FP8 E4M3 ("fn": no infinities, max 448), one byte per value.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *    enqueue work: they never synchronise with the host.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    failed check returns an error code and enqueues nothing.  Launch
+ *    failures return MOE_ERR_CUDA.  T == 0 is a valid no-op.
+ *  - Results are deterministic: the same inputs give bitwise the same
+ *    outputs on every call (no floating-point atomics; every sum has a
+ *    fixed order).
+ *  - Expert ids outside [0, E) contribute nothing to the output.
+ *  - Calls on the same stream may reuse the same workspace; calls that may
+ *    overlap (different streams) need separate workspaces.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad alignment     */
+    MOE_ERR_UNSUPPORTED = 2,   /* shape or mode outside what is implemented */
+    MOE_ERR_WORKSPACE = 3,     /* workspace missing or too small            */
+    MOE_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed       */
+    MOE_ERR_TIMEOUT = 5        /* reserved: a bounded device wait expired   */
+} moe_status_t;
+
+typedef enum {
+    MOE_W_BF16 = 0,            /* bf16 expert weights, bf16 activations      */
+    MOE_W_FP8_E4M3 = 1         /* e4m3 weights with fp32 per-(row,128) scales */
+} moe_wtype_t;
+
+/* Version of this ABI (incremented on any incompatible change). */
+MOE_API int moe_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+MOE_API const char *moe_status_string(moe_status_t status);
+
+/*
+ * Bytes of workspace needed by moe_experts_prefill (decode = 0) or
+ * moe_experts_decode (decode = 1) for these sizes.  Returns 0 when the sizes
+ * are invalid (the call itself then reports the error).
+ */
+MOE_API size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t wt, int decode);
+
+/*
+ * Routed-experts forward, prefill form: a grouped GEMM over experts
+ * (model card op "deepseek_ocr2_moe_experts").
+ *
+ *   hidden_states  [T,H]     bf16
+ *   gate_up_proj   [E,2F,H]  bf16 | e4m3; rows [0,F) of each expert are the
+ *                            gate projection, rows [F,2F) the up projection
+ *   down_proj      [E,H,F]   bf16 | e4m3
+ *   top_k_index    [T,K]     int32 expert ids
+ *   top_k_weights  [T,K]     fp32 router weights
+ *   top_k          K, 1 <= K <= 16
+ *   T >= 0, H % 128 == 0, F % 128 == 0, 1 <= E <= 1024
+ *   wt             weight dtype
+ *   gate_up_scale  [E,2F,H/128] fp32 (e4m3 only; NULL for bf16): the value of
+ *                  gate_up element (e,r,c) is e4m3(q) * gate_up_scale[e,r,c/128]
+ *   down_scale     [E,H,F/128]  fp32 (e4m3 only; NULL for bf16)
+ *   out            [T,H]     bf16, fully overwritten
+ *   workspace      device scratch of >= moe_experts_workspace_size(..., 0)
+ *                  bytes, 256-byte aligned; contents need no initialisation
+ *
+ * bf16 path: h = bf16(SiLU(g) * u) is stored in bf16 between the GEMMs;
+ * fp32 accumulation everywhere; the K contributions of a token are summed in
+ * k order in fp32 and rounded once to bf16.
+ * e4m3 path: hidden_states are quantised per 128 columns to e4m3 with a
+ * power-of-two scale (the rule of quantize_fp8_block128), h is rounded to
+ * bf16 and quantised the same way per 128 features, and each 128-long block
+ * of every dot product is scaled by its activation and weight scales.
+ * All pointers must be 16-byte aligned.
+ */
+MOE_API moe_status_t moe_experts_prefill(const void *hidden_states, const void *gate_up_proj,
+                                 const void *down_proj, const int32_t *top_k_index,
+                                 const float *top_k_weights, int top_k, int T, int H, int F,
+                                 int E, moe_wtype_t wt, const float *gate_up_scale,
+                                 const float *down_scale, void *out, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/*
+ * Routed-experts forward, decode form: a fused gather-GEMV for a few tokens
+ * (model card op "deepseek_ocr2_moe_experts_decode", n_tokens about 1-4).
+ * Same arguments, layouts and results as moe_experts_prefill, workspace from
+ * moe_experts_workspace_size(..., 1).  Tuned for T * K <= 64; larger calls
+ * are served by the prefill kernels (same results).
+ */
+MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_proj,
+                                const void *down_proj, const int32_t *top_k_index,
+                                const float *top_k_weights, int top_k, int T, int H, int F,
+                                int E, moe_wtype_t wt, const float *gate_up_scale,
+                                const float *down_scale, void *out, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
+ * Group-aware sigmoid top-k routing (layer table:
+ * moe_topk_sigmoid_routing_layer, num_groups=8, topk_group=4,
+ * routed_scaling_factor=2.5 for DeepSeek-V3).
+ *
+ *   logits [T,E] fp32, bias [E] fp32
+ *   s_e = sigmoid(logit_e) evaluated in double and rounded to fp32;
+ *   c_e = s_e + bias_e (fp32);
+ *   group score = sum of the two largest c_e of each of num_groups equal,
+ *   contiguous groups (the largest alone if a group has one expert);
+ *   the topk_group best groups are kept; top_k experts with the largest c_e
+ *   among the kept groups are chosen, best first;
+ *   top_k_weights[t,k] = (s_k / sum_j s_j) * routed_scaling_factor in fp32,
+ *   sum_j in selection order.  Equal scores rank the lower index first.
+ *   top_k_index [T,K] int32, top_k_weights [T,K] fp32 (outputs);
+ *   expert_offsets [E+1] int32 (optional output, may be NULL): exclusive
+ *   prefix sum of the number of slots routed to each expert.
+ * Limits: E % num_groups == 0, E <= 1024, num_groups <= 32,
+ * topk_group <= num_groups, top_k <= 16 and top_k <= experts in kept groups.
+ */
+MOE_API moe_status_t moe_route_sigmoid_grouped(const float *logits, const float *bias, int T, int E,
+                                       int num_groups, int topk_group, int top_k,
+                                       float routed_scaling_factor, int32_t *top_k_index,
+                                       float *top_k_weights, int32_t *expert_offsets,
+                                       void *stream);
+
+/*
+ * Block-wise FP8 quantisation (layer table: bf16_to_fp8_quantize, block 128).
+ *   x     [rows, cols] bf16, cols % 128 == 0
+ *   xq    [rows, cols] e4m3 (output)
+ *   scale [rows, cols/128] fp32 (output): per block of 128 values the
+ *         smallest power of two s = 2^k, -127 <= k <= 127, with
+ *         max|x| / s <= 448 (s = 1 for an all-zero block);
+ *         xq = e4m3(x / s), round-to-nearest-even, saturating at +-448.
+ */
+MOE_API moe_status_t quantize_fp8_block128(const void *x, int rows, int cols, void *xq, float *scale,
+                                   void *stream);
+
+/*
+ * Expert histogram and stable permutation of the T*K routing slots
+ * (slot = t*K + k), exposed for exact testing of the step the prefill path
+ * runs first.
+ *   counts  [E]    slots routed to each expert
+ *   offsets [E+1]  exclusive prefix sum of counts
+ *   perm    [T*K]  slot at each permuted position; positions of one expert
+ *                  hold its slots in ascending order; entries at positions
+ *                  >= offsets[E] (slots with ids outside [0,E)) are -1
+ *   inv     [T*K]  permuted position of each slot, -1 for ids outside [0,E)
+ *   workspace      >= moe_experts_workspace_size(T, 128, 128, E, K, MOE_W_BF16, 0)
+ */
+MOE_API moe_status_t moe_debug_permute(const int32_t *top_k_index, int T, int K, int E, int32_t *counts,
+                               int32_t *offsets, int32_t *perm, int32_t *inv, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,180 @@
+"""B200 (sm_100a) routed-experts MoE forward.
+
+Thin Python binding of ``libmoe_b200.so`` (C ABI in ``include/moe_b200.h``).
+Every function here only marshals arguments -- shapes, dtypes, device
+pointers, the current CUDA stream -- and calls the C entry point of the same
+name; all arithmetic runs in the library's CUDA kernels.  torch is used for
+device memory (outputs, workspaces) and streams only.
+
+The library must be built (``python -m mixture_experts_routed_expert_b200.build``
+or ``__graft_entry__.build()``); importing this package without it raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_W_BF16 = 0
+MOE_W_FP8_E4M3 = 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
+
+EXPORTS = ("moe_abi_version", "moe_status_string", "moe_experts_workspace_size",
+           "moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
+           "quantize_fp8_block128", "moe_debug_permute")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libmoe_b200.so is not built (run __graft_entry__.build() or "
+                          "python -m mixture_experts_routed_expert_b200.build)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+    L.moe_abi_version.restype = I
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_status_string.argtypes = [I]
+    L.moe_experts_workspace_size.restype = Z
+    L.moe_experts_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    fwd = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, Z, P]
+    L.moe_experts_prefill.argtypes = fwd
+    L.moe_experts_decode.argtypes = fwd
+    L.moe_route_sigmoid_grouped.argtypes = [P, P, I, I, I, I, I, F, P, P, P, P]
+    L.quantize_fp8_block128.argtypes = [P, I, I, P, P, P]
+    L.moe_debug_permute.argtypes = [P, I, I, I, P, P, P, P, P, Z, P]
+    for n in ("moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
+              "quantize_fp8_block128", "moe_debug_permute"):
+        getattr(L, n).restype = I
+    return L
+
+
+lib = _load()
+
+
+class MoEError(RuntimeError):
+    pass
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise MoEError("%s failed: %s" % (what, STATUS.get(rc, rc)))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _wtype(gate_up_proj):
+    if gate_up_proj.dtype == torch.bfloat16:
+        return MOE_W_BF16
+    if gate_up_proj.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return MOE_W_FP8_E4M3
+    raise TypeError("expert weights must be bf16 or e4m3 (uint8 / float8_e4m3fn)")
+
+
+def moe_experts_workspace_size(T, H, F, E, K, wtype=MOE_W_BF16, decode=False):
+    return int(lib.moe_experts_workspace_size(T, H, F, E, K, wtype, int(bool(decode))))
+
+
+def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
+             gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None):
+    T, H = hidden_states.shape
+    E, F2, H2 = gate_up_proj.shape
+    if H2 != H or down_proj.shape != (E, H, F2 // 2):
+        raise ValueError("shape mismatch: hidden %s gate_up %s down %s" % (
+            tuple(hidden_states.shape), tuple(gate_up_proj.shape), tuple(down_proj.shape)))
+    if tuple(top_k_index.shape) != (T, top_k) or tuple(top_k_weights.shape) != (T, top_k):
+        raise ValueError("top_k_index / top_k_weights must be [T, top_k]")
+    if top_k_index.dtype != torch.int32 or top_k_weights.dtype != torch.float32:
+        raise TypeError("top_k_index must be int32 and top_k_weights float32")
+    if hidden_states.dtype != torch.bfloat16:
+        raise TypeError("hidden_states must be bf16")
+    for t in (hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, gate_up_scale,
+              down_scale):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+    wt = _wtype(gate_up_proj)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
+    decode = name == "moe_experts_decode"
+    need = moe_experts_workspace_size(T, H, F2 // 2, E, top_k, wt, decode)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=hidden_states.device)
+    rc = getattr(lib, name)(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
+                            _ptr(top_k_index), _ptr(top_k_weights), top_k, T, H, F2 // 2, E, wt,
+                            _ptr(gate_up_scale), _ptr(down_scale), _ptr(out), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, name)
+    return out
+
+
+def moe_experts_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
+                        gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None):
+    """Routed-experts forward, grouped-GEMM form.  Returns out [T,H] bf16."""
+    return _forward("moe_experts_prefill", hidden_states, gate_up_proj, down_proj, top_k_index,
+                    top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream)
+
+
+def moe_experts_decode(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
+                       gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None):
+    """Routed-experts forward, fused gather-GEMV form for a few tokens."""
+    return _forward("moe_experts_decode", hidden_states, gate_up_proj, down_proj, top_k_index,
+                    top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream)
+
+
+def moe_route_sigmoid_grouped(logits, bias, num_groups, topk_group, top_k, routed_scaling_factor,
+                              top_k_index=None, top_k_weights=None, expert_offsets=None,
+                              want_offsets=False, stream=None):
+    """Group-aware sigmoid top-k routing.  Returns (top_k_index, top_k_weights[, offsets])."""
+    T, E = logits.shape
+    dev = logits.device
+    if top_k_index is None:
+        top_k_index = torch.empty(T, top_k, dtype=torch.int32, device=dev)
+    if top_k_weights is None:
+        top_k_weights = torch.empty(T, top_k, dtype=torch.float32, device=dev)
+    if want_offsets and expert_offsets is None:
+        expert_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    rc = lib.moe_route_sigmoid_grouped(_ptr(logits), _ptr(bias), T, E, num_groups, topk_group,
+                                       top_k, float(routed_scaling_factor), _ptr(top_k_index),
+                                       _ptr(top_k_weights), _ptr(expert_offsets), _stream(stream))
+    _check(rc, "moe_route_sigmoid_grouped")
+    if expert_offsets is not None:
+        return top_k_index, top_k_weights, expert_offsets
+    return top_k_index, top_k_weights
+
+
+def quantize_fp8_block128(x, xq=None, scale=None, stream=None):
+    """x [rows, cols] bf16 -> (xq [rows, cols] uint8 E4M3 codes, scale [rows, cols/128] f32)."""
+    rows, cols = x.shape
+    if xq is None:
+        xq = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(rows, cols // 128, dtype=torch.float32, device=x.device)
+    rc = lib.quantize_fp8_block128(_ptr(x), rows, cols, _ptr(xq), _ptr(scale), _stream(stream))
+    _check(rc, "quantize_fp8_block128")
+    return xq, scale
+
+
+def moe_debug_permute(top_k_index, E, workspace=None, stream=None):
+    """Expert counts, offsets, permutation and inverse of the routing slots."""
+    T, K = top_k_index.shape
+    dev = top_k_index.device
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(max(T * K, 1), dtype=torch.int32, device=dev)
+    inv = torch.empty(max(T * K, 1), dtype=torch.int32, device=dev)
+    need = moe_experts_workspace_size(T, 128, 128, E, K, MOE_W_BF16, False)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    rc = lib.moe_debug_permute(_ptr(top_k_index), T, K, E, _ptr(counts), _ptr(offsets), _ptr(perm),
+                               _ptr(inv), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "moe_debug_permute")
+    return counts, offsets, perm[:T * K], inv[:T * K]

@@ -1,0 +1,247 @@
+// api.cu -- the C ABI of libmoe_b200 (declared in include/moe_b200.h):
+// host-side validation, workspace layout and dispatch to the kernels.
+// Nothing here synchronises with the device or allocates device memory.
+#include <string.h>
+
+#include <algorithm>
+
+#include "internal.h"
+
+namespace moe {
+
+int num_sms() {
+    static int cache[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int &c = cache[dev & 63];
+    if (c == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        c = n;
+    }
+    return c;
+}
+
+namespace {
+
+struct Bump {
+    size_t off = 0;
+    size_t take(size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    }
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    cudaGetLastError();  // clear a sticky launch error so later calls can proceed
+    return e == cudaErrorInvalidValue ? MOE_ERR_INVALID_ARG : MOE_ERR_CUDA;
+}
+
+bool dims_ok(int64_t T, int H, int F, int E, int K) {
+    return T >= 0 && T <= (1 << 24) && H >= 128 && H % 128 == 0 && H <= 16384 && F >= 128 &&
+           F % 128 == 0 && F <= 16384 && E >= 1 && E <= 1024 && K >= 1 && K <= 16 &&
+           (int64_t)T * K < (1LL << 31) / 16;
+}
+
+}  // namespace
+
+Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t wt) {
+    const int64_t N = T * K;
+    const int64_t C = (N + kChunk - 1) / kChunk;
+    const size_t eb = (wt == MOE_W_BF16) ? 2 : 1;
+    Workspace L;
+    Bump b;
+    L.status = b.take(16);
+    L.chunk_hist = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(C, 1) * E);
+    L.slot_rank = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(C * kChunk, 1));
+    L.counts = b.take(sizeof(int32_t) * E);
+    L.offsets = b.take(sizeof(int32_t) * (E + 1));
+    L.tiles_g = b.take(sizeof(int32_t) * (E + 1));
+    L.tiles_d = b.take(sizeof(int32_t) * (E + 1));
+    L.perm = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(N, 1));
+    L.inv = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(N, 1));
+    L.xperm = b.take(eb * (size_t)N * H);
+    L.xscale = b.take(wt == MOE_W_BF16 ? 0 : sizeof(float) * (size_t)N * (H / 128));
+    L.h = b.take(eb * (size_t)N * F);
+    L.hscale = b.take(wt == MOE_W_BF16 ? 0 : sizeof(float) * (size_t)N * (F / 128));
+    L.y = b.take(sizeof(float) * (size_t)N * H);
+    L.total = b.off;
+    return L;
+}
+
+DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t wt) {
+    (void)H;
+    (void)E;
+    const size_t N = (size_t)T * K;
+    DecodeWorkspace L;
+    Bump b;
+    L.status = b.take(16);
+    L.h = b.take(2 * N * F);
+    L.hq = b.take(wt == MOE_W_BF16 ? 0 : N * F);
+    L.hscale = b.take(wt == MOE_W_BF16 ? 0 : sizeof(float) * N * (F / 128));
+    L.total = b.off;
+    return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+bool decode_fits(int T, int K) { return T <= kDecodeMaxT && T * K <= kDecodeMaxSlots; }
+
+moe_status_t check_common(const void *x, const void *gu, const void *dn, const int32_t *idx,
+                          const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
+                          const float *gus, const float *dns, const void *out) {
+    if (!dims_ok(T, H, F, E, K)) return MOE_ERR_INVALID_ARG;
+    if (wt != MOE_W_BF16 && wt != MOE_W_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !gu || !dn || !idx || !w || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(gu) || !aligned16(dn) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(idx) & 3) || (reinterpret_cast<uintptr_t>(w) & 3))
+        return MOE_ERR_INVALID_ARG;
+    if (wt == MOE_W_FP8_E4M3) {
+        if (!gus || !dns || !aligned16(gus) || !aligned16(dns)) return MOE_ERR_INVALID_ARG;
+    }
+    return MOE_OK;
+}
+
+moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const int32_t *idx,
+                         const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
+                         const float *gus, const float *dns, void *out, void *ws, size_t ws_bytes,
+                         cudaStream_t st) {
+    const Workspace L = prefill_workspace(T, H, F, E, K, wt);
+    if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
+    if (wt != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+    (void)gus;
+    (void)dns;
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    const int64_t N = (int64_t)T * K;
+    cudaError_t e = launch_permute(idx, N, E, wsb, L, st);
+    if (e == cudaSuccess) e = launch_gather(x, idx, N, K, H, E, wt, wsb, L, st);
+    if (e == cudaSuccess) e = launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st);
+    if (e == cudaSuccess) e = launch_combine(idx, T, H, E, K, wsb, L, out, st);
+    return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return 1; }
+
+const char *moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t wt, int decode) {
+    if (!dims_ok(T, H, F, E, K)) return 0;
+    if (decode && decode_fits(T, K)) return decode_workspace(T, H, F, E, K, wt).total;
+    return prefill_workspace(T, H, F, E, K, wt).total;
+}
+
+moe_status_t moe_experts_prefill(const void *hidden_states, const void *gate_up_proj,
+                                 const void *down_proj, const int32_t *top_k_index,
+                                 const float *top_k_weights, int top_k, int T, int H, int F,
+                                 int E, moe_wtype_t wt, const float *gate_up_scale,
+                                 const float *down_scale, void *out, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                  top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
+                                  out);
+    if (s != MOE_OK || T == 0) return s;
+    return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
+                       T, H, F, E, wt, gate_up_scale, down_scale, out, workspace, workspace_bytes,
+                       (cudaStream_t)stream);
+}
+
+moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_proj,
+                                const void *down_proj, const int32_t *top_k_index,
+                                const float *top_k_weights, int top_k, int T, int H, int F, int E,
+                                moe_wtype_t wt, const float *gate_up_scale,
+                                const float *down_scale, void *out, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                  top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
+                                  out);
+    if (s != MOE_OK || T == 0) return s;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (!decode_fits(T, top_k))
+        return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
+                           top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
+                           workspace_bytes, st);
+    const DecodeWorkspace L = decode_workspace(T, H, F, E, top_k, wt);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return MOE_ERR_WORKSPACE;
+    if (wt != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+    return from_cuda(launch_decode_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                        top_k_weights, T, H, F, E, top_k,
+                                        static_cast<uint8_t *>(workspace), L, out, st));
+}
+
+moe_status_t moe_route_sigmoid_grouped(const float *logits, const float *bias, int T, int E,
+                                       int num_groups, int topk_group, int top_k,
+                                       float routed_scaling_factor, int32_t *top_k_index,
+                                       float *top_k_weights, int32_t *expert_offsets,
+                                       void *stream) {
+    if (T < 0 || E < 1 || E > 1024 || num_groups < 1 || num_groups > 32 || E % num_groups ||
+        topk_group < 1 || topk_group > num_groups || top_k < 1 || top_k > 16 ||
+        top_k > topk_group * (E / num_groups))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) {
+        if (expert_offsets) return from_cuda(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), (cudaStream_t)stream));
+        return MOE_OK;
+    }
+    if (!logits || !bias || !top_k_index || !top_k_weights) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_route(logits, bias, T, E, num_groups, topk_group, top_k,
+                                  routed_scaling_factor, top_k_index, top_k_weights, expert_offsets,
+                                  (cudaStream_t)stream));
+}
+
+moe_status_t quantize_fp8_block128(const void *x, int rows, int cols, void *xq, float *scale,
+                                   void *stream) {
+    if (rows < 0 || cols <= 0 || cols % 128) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!x || !xq || !scale || !aligned16(x) || !aligned16(xq) ||
+        (reinterpret_cast<uintptr_t>(scale) & 3))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_quantize(x, rows, cols, xq, scale, (cudaStream_t)stream));
+}
+
+moe_status_t moe_debug_permute(const int32_t *top_k_index, int T, int K, int E, int32_t *counts,
+                               int32_t *offsets, int32_t *perm, int32_t *inv, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    if (!dims_ok(T, 128, 128, E, K)) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || (T > 0 && (!top_k_index || !perm || !inv)))
+        return MOE_ERR_INVALID_ARG;
+    const Workspace L = prefill_workspace(T, 128, 128, E, K, MOE_W_BF16);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return MOE_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int64_t N = (int64_t)T * K;
+    if (N == 0) {
+        cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
+        return from_cuda(e);
+    }
+    cudaError_t e = launch_permute(top_k_index, N, E, ws, L, st);
+    if (e == cudaSuccess) e = launch_debug_outputs(top_k_index, N, E, ws, L, counts, offsets, perm, inv, st);
+    return from_cuda(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,361 @@
+// gemm_bf16.cu -- S4 and S5 of the prefill path: grouped GEMMs over experts on
+// the 5th-generation tensor cores (tcgen05, accumulators in TMEM, operands
+// staged by TMA).
+//
+// S4 (gate_up, fused SiLU * up):  for the rows r of expert e (routed slots in
+//   expert order),  h[r, f] = bf16( SiLU(G_e[f] . x_r) * (U_e[f] . x_r) ).
+// S5 (down, fused router-weight scale):  y[s, j] = w[s] * (D_e[j] . h[r]),
+//   s = perm[r] the original slot t*K+k; rows are written by slot so that the
+//   combine can sum a token's K rows in k order.
+// ("deepseek-ocr2-moe-experts" model card, description: grouped GEMM for
+// prefill shapes, plain SiLU SwiGLU, router-weight scale + scatter-add.)
+//
+// Tile = (expert e, 128 weight rows, up to BN routed rows), "swap-AB": the
+// weights sit on the MMA M=128 side and the routed rows on N, so small
+// experts waste no MMA rows; N is rounded up to 16 per tile.
+// Persistent: one CTA per SM walks the tile list (the tile count is read on
+// the device; the host never synchronises).  Warp roles:
+//   warp 0     TMA producer (4-stage shared-memory ring)
+//   warp 1     TMEM allocation + MMA issue (one thread)
+//   warps 2-5  epilogue: TMEM -> registers -> global (double-buffered TMEM)
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kBK = 64;           // bf16 elements per k-block = one 128-byte swizzle row
+constexpr int kBoxRows = 32;      // routed rows per TMA box of the B operand
+constexpr int kThreads = 192;
+
+template <bool GATE_UP>
+struct Cfg {
+    static constexpr int BN = GATE_UP ? kBNGateUp : kBNDown;
+    static constexpr int NUM_A = GATE_UP ? 2 : 1;      // gate and up weight tiles
+    static constexpr int A_BYTES = kBM * 128;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    static constexpr int ACC_COLS = NUM_A * BN;        // TMEM columns per accumulator set
+    static constexpr int NUM_ACC = 512 / ACC_COLS;     // accumulator sets (2)
+    static constexpr int RING_BYTES = kStages * STAGE_BYTES;
+    static size_t smem_bytes(int E) { return RING_BYTES + 1024 + 1024 + 2 * sizeof(int) * (E + 1); }
+};
+
+struct GemmArgs {
+    const int32_t *offsets;      // [E+1] first routed row of each expert
+    const int32_t *tiles;        // [E+1] prefix sum of row tiles per expert
+    int E, MT, KB;               // experts, weight-row tiles per expert, k-blocks
+    int a_rows_per_expert;       // 2F (gate_up) or H (down)
+    int up_offset;               // F: row offset of the up half (gate_up)
+    __nv_bfloat16 *h;            // gate_up output [N][F]
+    int F;
+    float *y;                    // down output [T*K][H]
+    int H;
+    const int32_t *perm;         // [N] routed row -> slot
+    const float *topw;           // [T*K] router weights
+    int32_t *status;
+};
+
+struct Tile {
+    int e, m, row0, nrows;
+};
+
+__device__ __forceinline__ Tile decode_tile(int w, const int32_t *s_off, const int32_t *s_tiles,
+                                            int E, int MT, int BN) {
+    int lo = 0, hi = E;  // s_tiles[lo]*MT <= w < s_tiles[hi]*MT
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_tiles[mid] * MT <= w) lo = mid; else hi = mid;
+    }
+    Tile t;
+    t.e = lo;
+    const int nt = s_tiles[lo + 1] - s_tiles[lo];
+    const int local = w - s_tiles[lo] * MT;
+    t.m = local / nt;
+    const int n = local - t.m * nt;
+    t.row0 = s_off[lo] + n * BN;
+    t.nrows = min(BN, s_off[lo + 1] - t.row0);
+    return t;
+}
+
+template <bool GATE_UP>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmArgs args) {
+    using C = Cfg<GATE_UP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ring = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::RING_BYTES);
+    uint64_t *empty = full + kStages;
+    uint64_t *tfull = empty + kStages;
+    uint64_t *tempty = tfull + C::NUM_ACC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + C::NUM_ACC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int32_t *s_off = reinterpret_cast<int32_t *>(smem + C::RING_BYTES + 1024);
+    int32_t *s_tiles = s_off + (args.E + 1);
+
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < C::NUM_ACC; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    pdl_wait();  // routed rows, offsets and tiles come from the previous kernels
+    for (int i = threadIdx.x; i <= args.E; i += blockDim.x) {
+        s_off[i] = args.offsets[i];
+        s_tiles[i] = args.tiles[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = s_tiles[args.E] * args.MT;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            int armed[kStages];
+#pragma unroll
+            for (int s = 0; s < kStages; ++s) armed[s] = -1;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, C::BN);
+                const int nbox = (t.nrows + kBoxRows - 1) / kBoxRows;
+                const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * kBoxRows * 128;
+                const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
+                for (int kb = 0; kb < args.KB; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t *sA = ring + stage * C::STAGE_BYTES;
+                    uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    armed[stage] = (int)phase;
+                    tma_load_2d(sA, &tmA, &full[stage], kb * kBK, arow, pol_w);
+                    if (GATE_UP)
+                        tma_load_2d(sA + C::A_BYTES, &tmA, &full[stage], kb * kBK,
+                                    arow + args.up_offset, pol_w);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(sB + b * kBoxRows * 128, &tmB, &full[stage], kb * kBK,
+                                    t.row0 + b * kBoxRows, pol_x);
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+            }
+            // drain: every armed stage must have landed before the CTA exits
+            volatile int never = 0;
+            for (int s = 0; s < kStages; ++s)
+                if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
+                    atomicOr(args.status, DEV_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer ------
+        if (lane == 0) {
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, C::BN);
+                const int N = (t.nrows + 15) & ~15;
+                const uint32_t idesc = idesc_bf16(kBM, N);
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem_base + acc * C::ACC_COLS;
+                for (int kb = 0; kb < args.KB; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(ring + stage * C::STAGE_BYTES);
+                    const uint64_t da = sdesc_sw128(sa);
+                    const uint64_t da2 = sdesc_sw128(sa + C::A_BYTES);
+                    const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        const uint32_t accum = (kb | k) != 0;
+                        mma_bf16_ss(d, da + 2 * k, db + 2 * k, idesc, accum);
+                        if (GATE_UP) mma_bf16_ss(d + C::BN, da2 + 2 * k, db + 2 * k, idesc, accum);
+                    }
+                    mma_commit(&empty[stage]);
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1; }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue --------
+        const int eg = warp & 3;                // TMEM lanes [32*eg, 32*eg+32)
+        const int row = eg * 32 + lane;         // weight row inside the tile
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, C::BN);
+            if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) {
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + acc * C::ACC_COLS;
+            for (int c0 = 0; c0 < t.nrows; c0 += 32) {
+                uint32_t g[32];
+                tmem_ld32(tb + c0, g);
+                if (GATE_UP) {
+                    uint32_t u[32];
+                    tmem_ld32(tb + C::BN + c0, u);
+                    tmem_ld_wait();
+                    __nv_bfloat16 *hp = args.h + (size_t)(t.row0 + c0) * args.F + t.m * kBM + row;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        if (c0 + j < t.nrows) {
+                            const float gv = __uint_as_float(g[j]);
+                            hp[(size_t)j * args.F] = __float2bfloat16_rn(silu_f(gv) * __uint_as_float(u[j]));
+                        }
+                    }
+                } else {
+                    tmem_ld_wait();
+                    const int c = c0 + lane;
+                    const int my_slot = (c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
+                    const float my_w = (c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
+                    float *yp = args.y + t.m * kBM + row;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                        const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                        if (c0 + j < t.nrows) yp[(size_t)slot * args.H] = wj * __uint_as_float(g[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            if (++acc == C::NUM_ACC) { acc = 0; acc_phase ^= 1; }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// Row-major [rows, cols] matrix, box = box_rows x 128 bytes, 128-byte swizzle.
+bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int elem_bytes, const void *ptr,
+               uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool GATE_UP>
+cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmArgs &args,
+                       cudaStream_t st) {
+    using C = Cfg<GATE_UP>;
+    const size_t smem = C::smem_bytes(args.E);
+    static int attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16<GATE_UP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)C::smem_bytes(1024));
+        if (e != cudaSuccess) return e;
+        attr_done[dev & 63] = 1;
+    }
+    return launch_k(grouped_gemm_bf16<GATE_UP>, dim3(num_sms()), dim3(kThreads), smem, st, true, a,
+                    b, args);
+}
+
+}  // namespace
+
+cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float *topw, int64_t T,
+                              int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
+                              cudaStream_t st) {
+    const uint64_t N = (uint64_t)T * K;
+    CUtensorMap ta, tb, tc, td;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_tmap(&ta, BF, 2, gate_up, (uint64_t)E * 2 * F, H, kBM) ||
+        !make_tmap(&tb, BF, 2, ws + L.xperm, N, H, kBoxRows) ||
+        !make_tmap(&tc, BF, 2, down, (uint64_t)E * H, F, kBM) ||
+        !make_tmap(&td, BF, 2, ws + L.h, N, F, kBoxRows))
+        return cudaErrorInvalidValue;
+    GemmArgs g = {};
+    g.offsets = (const int32_t *)(ws + L.offsets);
+    g.E = E;
+    g.perm = (const int32_t *)(ws + L.perm);
+    g.topw = topw;
+    g.status = (int32_t *)(ws + L.status);
+    g.h = (__nv_bfloat16 *)(ws + L.h);
+    g.y = (float *)(ws + L.y);
+    g.F = F;
+    g.H = H;
+
+    GemmArgs a1 = g;
+    a1.tiles = (const int32_t *)(ws + L.tiles_g);
+    a1.MT = F / kBM;
+    a1.KB = H / kBK;
+    a1.a_rows_per_expert = 2 * F;
+    a1.up_offset = F;
+    cudaError_t err = launch_one<true>(ta, tb, a1, st);
+    if (err != cudaSuccess) return err;
+
+    GemmArgs a2 = g;
+    a2.tiles = (const int32_t *)(ws + L.tiles_d);
+    a2.MT = H / kBM;
+    a2.KB = F / kBK;
+    a2.a_rows_per_expert = H;
+    a2.up_offset = 0;
+    return launch_one<false>(tc, td, a2, st);
+}
+
+}  // namespace moe

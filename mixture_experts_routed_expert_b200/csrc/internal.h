@@ -1,0 +1,96 @@
+// internal.h -- host-side declarations shared by the translation units of
+// libmoe_b200 (launchers, workspace layout, tile configuration).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+// ---- grouped-GEMM tiling (shared by the scheduler in the permute kernels) --
+constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBNGateUp = 128;    // routed rows (tokens) per gate_up tile
+constexpr int kBNDown = 256;      // routed rows per down tile
+constexpr int kChunk = 2048;      // routing slots per histogram block
+
+// ---- workspace layout ------------------------------------------------------
+struct Workspace {
+    size_t status;        // int32 device status word
+    size_t chunk_hist;    // [C][E] int32: per-chunk counts, then per-chunk bases
+    size_t slot_rank;     // [N] int32 rank of a slot among its chunk's slots of one expert
+    size_t counts;        // [E] int32
+    size_t offsets;       // [E+1] int32
+    size_t tiles_g;       // [E+1] int32 prefix of gate_up row tiles per expert
+    size_t tiles_d;       // [E+1] int32 prefix of down row tiles per expert
+    size_t perm;          // [N] int32
+    size_t inv;           // [N] int32
+    size_t xperm;         // [N][H] bf16 | e4m3
+    size_t xscale;        // [N][H/128] f32 (e4m3 only)
+    size_t h;             // [N][F] bf16 | e4m3
+    size_t hscale;        // [N][F/128] f32 (e4m3 only)
+    size_t y;             // [N][H] f32 (weighted down-projection rows, by slot)
+    size_t total;
+};
+Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t wt);
+
+struct DecodeWorkspace {
+    size_t status;
+    size_t h;             // [T*K][F] bf16
+    size_t hq;            // [T*K][F] e4m3 + scales (e4m3 path)
+    size_t hscale;
+    size_t total;
+};
+DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t wt);
+
+constexpr int kDecodeMaxSlots = 64;  // T*K served by the decode kernels
+constexpr int kDecodeMaxT = 16;
+
+// ---- launchers (return cudaSuccess or the launch error) --------------------
+int num_sms();
+
+cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, uint8_t *ws,
+                           const Workspace &L, cudaStream_t st);
+cudaError_t launch_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H, int E,
+                          moe_wtype_t wt, uint8_t *ws, const Workspace &L, cudaStream_t st);
+cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, const uint8_t *ws,
+                                 const Workspace &L, int32_t *counts, int32_t *offsets,
+                                 int32_t *perm, int32_t *inv, cudaStream_t st);
+cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float *topw, int64_t T,
+                              int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
+                              cudaStream_t st);
+cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, const uint8_t *ws,
+                           const Workspace &L, void *out, cudaStream_t st);
+cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *down,
+                               const int32_t *idx, const float *w, int T, int H, int F, int E,
+                               int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
+                               cudaStream_t st);
+cudaError_t launch_quantize(const void *x, int64_t rows, int cols, void *xq, float *scale,
+                            cudaStream_t st);
+cudaError_t launch_route(const float *logits, const float *bias, int64_t T, int E, int num_groups,
+                         int topk_group, int top_k, float scale, int32_t *idx, float *w,
+                         int32_t *offsets, cudaStream_t st);
+
+// cudaLaunchKernelEx with optional programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace moe

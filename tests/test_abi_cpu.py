@@ -1,0 +1,64 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host (no GPU needed: validation happens before
+any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+@pytest.fixture(scope="module")
+def mod():
+    import mixture_experts_routed_expert_b200 as m
+    return m
+
+
+def test_exports_match_header(mod):
+    decl = set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(", open(HEADER).read()))
+    assert decl == set(mod.EXPORTS)
+    for name in decl:
+        assert hasattr(mod.lib, name), name
+    assert mod.lib.moe_abi_version() == 1
+    assert mod.lib.moe_status_string(3) == b"MOE_ERR_WORKSPACE"
+
+
+def test_workspace_sizes(mod):
+    ws = mod.moe_experts_workspace_size
+    assert ws(2048, 1280, 896, 64, 6) > 2048 * 6 * (1280 * 2 + 896 * 2 + 1280 * 4)
+    assert ws(1, 1280, 896, 64, 6, decode=True) >= 6 * 896 * 2
+    assert ws(4, 1280, 896, 64, 6, decode=True) < ws(4, 1280, 896, 64, 6)
+    assert ws(16, 100, 896, 64, 6) == 0          # H % 128 != 0
+    assert ws(16, 1280, 896, 0, 6) == 0          # E == 0
+    assert ws(16, 1280, 896, 64, 17) == 0        # K > 16
+
+
+def test_host_validation_without_gpu(mod):
+    L = mod.lib
+    N = None
+    # T == 0 is a valid no-op
+    assert L.moe_experts_prefill(N, N, N, N, N, 6, 0, 1280, 896, 64, 0, N, N, N, N, 0, N) == 0
+    # bad sizes
+    assert L.moe_experts_prefill(N, N, N, N, N, 6, 4, 1000, 896, 64, 0, N, N, N, N, 0, N) == 1
+    assert L.moe_experts_decode(N, N, N, N, N, 0, 4, 1280, 896, 64, 0, N, N, N, N, 0, N) == 1
+    # null tensors
+    assert L.moe_experts_prefill(N, N, N, N, N, 6, 4, 1280, 896, 64, 0, N, N, N, N, 0, N) == 1
+    # misaligned pointer
+    p = ctypes.c_void_p(0x1000)
+    q = ctypes.c_void_p(0x1001)
+    assert L.moe_experts_prefill(q, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, p, p, 1 << 30, N) == 1
+    # FP8 without scales
+    assert L.moe_experts_prefill(p, p, p, p, p, 6, 4, 1280, 896, 64, 1, N, N, p, p, 1 << 30, N) == 1
+    # workspace too small / missing
+    assert L.moe_experts_prefill(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, p, p, 16, N) == 3
+    assert L.moe_experts_prefill(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, p, N, 0, N) == 3
+    # router limits
+    assert L.moe_route_sigmoid_grouped(p, p, 4, 256, 7, 4, 8, 2.5, p, p, N, N) == 1
+    assert L.moe_route_sigmoid_grouped(p, p, 4, 256, 8, 9, 8, 2.5, p, p, N, N) == 1
+    assert L.moe_route_sigmoid_grouped(p, p, 0, 256, 8, 4, 8, 2.5, p, p, N, N) == 0
+    # quantiser limits
+    assert L.quantize_fp8_block128(p, 4, 100, p, p, N) == 1
+    assert L.quantize_fp8_block128(p, 0, 128, p, p, N) == 0
