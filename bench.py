@@ -1,0 +1,399 @@
+#!/usr/bin/env python3
+"""Benchmark of the routed-experts MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one routed-experts MoE layer on the OCR-2 decode shape
+(T=1 token, H=1280, F=896, E=64 experts, top-6, bf16; synthetic seeded
+inputs, all 64 experts' weights resident in HBM), run through the C ABI of
+libmoe_b200.so and replayed from a CUDA graph.  L2 is flushed (a 512 MiB
+buffer is written) before every timed step, outside the timed interval.
+Each step is timed with CUDA events on the launching stream; the JSON line
+reports the sum over the K timed steps, max over ranks.
+
+Metric: microseconds per MoE layer (lower is better).  The line also carries
+a roofline entry (HBM GB/s on the touched expert weights against the measured
+copy bandwidth), the CPU oracle timed on a bounded sample of the same
+workload, an end-to-end figure (host buffers, copies inside the timed
+region), SM clocks sampled during the timed region, and a breakdown with the
+other decode sizes and the OCR-2 prefill (T=2048) layer.
+
+With N > 1 (torchrun), every rank runs an independent replica of the same
+workload on its own GPU (the layer has no data-path collective on one GPU's
+worth of experts); value = summed time of the slowest rank / layers done by
+all ranks.
+
+--impl reference times the CPU oracle (the plain C reference of the layer)
+on the host cores for the same metric and workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PAGES_DECODE_T1_US = 191.0       # model card, GB10 decode latency (context only)
+METRIC = "us_per_moe_layer"
+FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------- workloads --
+
+def touched_bytes_bf16(idx, H, F):
+    n = len(set(int(e) for e in idx.reshape(-1).tolist() if e >= 0))
+    return n, n * 3 * H * F * 2
+
+
+def layer_alg(idx, T, H, F, K):
+    """Algorithmic bytes (touched expert weights + x + out + idx + w) and flops."""
+    n_touched, wbytes = touched_bytes_bf16(idx, H, F)
+    io = T * H * 2 * 2 + T * K * 8
+    return dict(touched_experts=n_touched, bytes=wbytes + io, flops=6 * T * K * H * F)
+
+
+# ------------------------------------------------------------------ clocks ----
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 6]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[0]) for r in rows if r[0].strip().replace(".", "").isdigit()]
+        smax = max(float(r[1]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" == r[3 + i].strip()})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------- ours -----
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_routed_expert_b200 as moe
+    from mixture_experts_routed_expert_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks = load_peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream()
+
+    def time_graph(fn, steps, warmup):
+        """Capture fn() in a CUDA graph; replay with an L2 flush before each
+        timed replay; returns per-step device times in microseconds."""
+        fn()  # first call outside capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(warmup):
+            flush.fill_(1)
+            g.replay()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            g.replay()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return [a.elapsed_time(b) * 1e3 for a, b in evs], g
+
+    def time_eager(fn, steps, warmup):
+        for _ in range(warmup):
+            flush.fill_(1)
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            fn()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) * 1e3 for a, b in evs]
+
+    # ---- headline workload: OCR-2 decode, T=1 ----------------------------
+    base = inputs.ocr2_layer(1, seed=0, device=dev)
+    H, F, E, K = 1280, 896, 64, 6
+
+    def make_call(T, seed, fn=moe.moe_experts_decode, decode=True):
+        lay = inputs.ocr2_layer(T, seed=seed, device=dev, weights_from=base)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(moe.moe_experts_workspace_size(T, H, F, E, K, 0, decode), 256),
+                         dtype=torch.uint8, device=dev)
+        call = lambda: fn(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K, out=out, workspace=ws)
+        return lay, out, ws, call
+
+    lay1, out1, ws1, call1 = make_call(1, 1)
+    alg1 = layer_alg(lay1.idx.cpu().numpy(), 1, H, F, K)
+    with ClockSampler(local) as clk:
+        times, graph1 = time_graph(call1, args.steps, args.warmup)
+    clocks = clk.summary()
+    total_us = max_over_ranks(sum(times))
+    per_layer_us = total_us / (args.steps * world)
+    layer_us = total_us / args.steps
+    achieved = alg1["bytes"] / (layer_us * 1e-6) / 1e9
+    launches_per_step = 2
+
+    # ---- end to end through the C ABI with host buffers -------------------
+    xh = lay1.x.cpu().pin_memory()
+    ih = lay1.idx.cpu().pin_memory()
+    wh = lay1.w.cpu().pin_memory()
+    oh = torch.empty_like(out1, device="cpu").pin_memory()
+    xd, idd, wd = torch.empty_like(lay1.x), torch.empty_like(lay1.idx), torch.empty_like(lay1.w)
+
+    def e2e_call():
+        xd.copy_(xh, non_blocking=True)
+        idd.copy_(ih, non_blocking=True)
+        wd.copy_(wh, non_blocking=True)
+        moe.moe_experts_decode(xd, lay1.gate_up, lay1.down, idd, wd, K, out=out1, workspace=ws1)
+        oh.copy_(out1, non_blocking=True)
+
+    e2e_times = time_eager(e2e_call, args.steps, args.warmup)
+    e2e_us = max_over_ranks(sum(e2e_times)) / (args.steps * world)
+    h2d = xh.numel() * 2 + ih.numel() * 4 + wh.numel() * 4
+    d2h = oh.numel() * 2
+
+    # ---- breakdown: other decode sizes, eager decode, OCR-2 prefill ---------
+    breakdown = {}
+    eager1 = time_eager(call1, args.steps, args.warmup)
+    breakdown["decode_T1_eager_us"] = round(float(np.mean(eager1)), 2)
+    for T in (2, 4, 8):
+        lay, out, ws, call = make_call(T, T)
+        t, g = time_graph(call, args.steps, args.warmup)
+        a = layer_alg(lay.idx.cpu().numpy(), T, H, F, K)
+        us = float(np.mean(t))
+        breakdown["decode_T%d" % T] = dict(us=round(us, 2), touched_experts=a["touched_experts"],
+                                           gbs=round(a["bytes"] / us / 1e3, 1),
+                                           hbm_frac=round(a["bytes"] / us / 1e3 / peaks["hbm"], 3))
+        del g
+    lay, out, ws, call = make_call(2048, 2048, fn=moe.moe_experts_prefill, decode=False)
+    t, g = time_graph(call, args.steps, args.warmup)
+    a = layer_alg(lay.idx.cpu().numpy(), 2048, H, F, K)
+    us = float(np.mean(t))
+    t_hbm = a["bytes"] / (peaks["hbm"] * 1e3)
+    t_tc = a["flops"] / (peaks["bf16"] * 1e6)
+    breakdown["prefill_T2048"] = dict(
+        us=round(us, 2), tflops=round(a["flops"] / us / 1e6, 1), gbs=round(a["bytes"] / us / 1e3, 1),
+        tc_frac=round(t_tc / us, 3), hbm_frac=round(t_hbm / us, 3),
+        roofline_frac=round(max(t_hbm, t_tc) / us, 3), bound="hbm" if t_hbm > t_tc else "tensor")
+    del g
+
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "decode_ocr2_T1_traffic.json")
+    if os.path.exists(tfile):
+        tj = json.load(open(tfile))
+        src = os.path.join(ROOT, "mixture_experts_routed_expert_b200", "csrc", "decode.cu")
+        if tj.get("source_sha256") == hashlib.sha256(open(src, "rb").read()).hexdigest():
+            traffic = tj.get("dram_bytes_per_launch")
+
+    result = {
+        "metric": METRIC, "value": round(per_layer_us, 3), "unit": "us/layer",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(layer_us / 1e3, 6), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": round(per_layer_us / PAGES_DECODE_T1_US, 4),
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) hidden, N(0,0.02^2) weights, softmax top-6 routing)",
+        "config": {"workload": "OCR-2 routed experts, decode T=1 (H=1280 F=896 E=64 K=6, bf16)",
+                   "global_batch": world, "seq_len": 1, "parallelism": "replicas%d" % world,
+                   "l2": "flushed (512 MiB write) before every timed step",
+                   "timing": "CUDA graph replay of the C-ABI call, CUDA events"},
+        "roofline": {"bound": "hbm", "kernel": "decode_up_bf16 + decode_down_bf16 (PDL chain)",
+                     "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm"], 4), "traffic": traffic,
+                     "algorithmic_bytes": alg1["bytes"], "peak_source": peaks["source"]},
+        "e2e": {"value": round(e2e_us, 3), "unit": "us/layer", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "breakdown": breakdown,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        del graph1
+        dist.destroy_process_group()
+
+
+def run_only(args):
+    """W + K eager calls of one workload with an L2 flush before each, no
+    timing report: the command that profiler captures are taken on."""
+    import torch
+
+    import mixture_experts_routed_expert_b200 as moe
+    from mixture_experts_routed_expert_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    T = {"decode1": 1, "decode4": 4, "prefill2048": 2048}[args.only]
+    fn = moe.moe_experts_prefill if args.only.startswith("prefill") else moe.moe_experts_decode
+    lay = inputs.ocr2_layer(T, seed=T, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = None
+    for i in range(args.warmup + args.steps):
+        flush.fill_(i & 0xFF)
+        out = fn(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, 6)
+    torch.cuda.synchronize()
+    print("ok", args.only, float(out.float().abs().sum()))
+
+
+# ------------------------------------------------------------- reference -----
+
+def cpu_baseline(budget_s=12.0):
+    """The oracle (plain C, fp64, OpenMP over tokens) on the host cores, on a
+    bounded sample of decode layers of the same workload; us per layer."""
+    import torch
+
+    import oracle
+    from mixture_experts_routed_expert_b200 import inputs
+
+    lay = inputs.ocr2_layer(1, seed=1, device="cpu")
+    gu = inputs.bf16_bits(lay.gate_up)
+    dn = inputs.bf16_bits(lay.down)
+    x, idx, w = inputs.bf16_bits(lay.x), inputs.np32(lay.idx), inputs.np32(lay.w)
+    oracle.moe_forward_bf16(x, gu, dn, idx, w)       # warm
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.moe_forward_bf16(x, gu, dn, idx, w)
+        n += 1
+        if time.perf_counter() - t0 > budget_s or n >= 200:
+            break
+    el = time.perf_counter() - t0
+    # the oracle parallelises over tokens: a T=1 layer runs on one thread
+    return {"value": round(el / n * 1e6, 1), "unit": "us/layer", "cores": min(oracle.num_threads(), 1),
+            "kind": "oracle",
+            "sample": "%d decode layers (T=1) of the OCR-2 workload, %.1f s wall" % (n, el)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    times = []
+    import oracle
+    from mixture_experts_routed_expert_b200 import inputs
+    lay = inputs.ocr2_layer(1, seed=1, device="cpu")
+    gu, dn = inputs.bf16_bits(lay.gate_up), inputs.bf16_bits(lay.down)
+    x, idx, w = inputs.bf16_bits(lay.x), inputs.np32(lay.idx), inputs.np32(lay.w)
+    for _ in range(args.warmup):
+        oracle.moe_forward_bf16(x, gu, dn, idx, w)
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.moe_forward_bf16(x, gu, dn, idx, w)
+        times.append((time.perf_counter() - t0) * 1e6)
+    v = float(np.sum(times)) / args.steps
+    cores = min(oracle.num_threads(), 1)   # parallel over tokens; T=1
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": "us/layer",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(v / 1e3, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": round(v / PAGES_DECODE_T1_US, 4), "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "OCR-2 routed experts, decode T=1 (H=1280 F=896 E=64 K=6, bf16)",
+                   "global_batch": 1, "seq_len": 1, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(v, 1), "unit": "us/layer", "cores": cores, "kind": "oracle",
+                         "sample": "%d decode layers (T=1), one per step" % args.steps},
+        "e2e": {"value": round(v, 1), "unit": "us/layer", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048"], default=None,
+                    help="run just W+K eager calls of one workload (for profiler captures)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.only:
+        run_only(args)
+    elif args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

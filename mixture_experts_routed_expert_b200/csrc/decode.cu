@@ -22,34 +22,66 @@ namespace {
 
 constexpr int kUpWarps = 16;
 constexpr int kDownWarps = 16;
-constexpr int kSlotGroup = 4;   // slots of one expert handled per weight pass
-constexpr int kChunkVec = 4;    // 16-byte vectors per lane kept in flight per row
+constexpr int kSlotGroup = 1;   // slots of one expert handled per pass over the loaded rows
 
 // Distinct experts of the T*K slots, in order of first appearance, with the
-// slots of each in ascending order.  Built by one thread.
+// slots of each in ascending order.  Built cooperatively by the first
+// kDecodeMaxSlots threads of the block (one slot each); every thread must call
+// it (it contains __syncthreads).
 struct Touched {
     int n;
     int expert[kDecodeMaxSlots];
     int start[kDecodeMaxSlots + 1];
     int slot[kDecodeMaxSlots];
+    int e_of[kDecodeMaxSlots];     // expert id of each slot (-1 when out of range)
+    int u_of[kDecodeMaxSlots];     // touched index of each slot
 };
 
 __device__ void build_touched(const int32_t *__restrict__ idx, int TK, int E, Touched &u) {
-    int n = 0, m = 0;
-    for (int s = 0; s < TK; ++s) {
-        const int e = idx[s];
-        if (e < 0 || e >= E) continue;
-        bool seen = false;
-        for (int i = 0; i < n; ++i) seen |= (u.expert[i] == e);
-        if (!seen) u.expert[n++] = e;
+    __shared__ int is_first[kDecodeMaxSlots];
+    const int s = threadIdx.x;
+    if (s < TK) {
+        const int e = __ldg(idx + s);
+        u.e_of[s] = (e >= 0 && e < E) ? e : -1;
     }
-    for (int i = 0; i < n; ++i) {
-        u.start[i] = m;
-        for (int s = 0; s < TK; ++s)
-            if (idx[s] == u.expert[i]) u.slot[m++] = s;
+    __syncthreads();
+    int e = -1, first = -1;
+    if (s < TK) {
+        e = u.e_of[s];
+        if (e >= 0) {
+            first = s;
+            for (int q = 0; q < s; ++q)
+                if (u.e_of[q] == e) { first = q; break; }
+        }
+        is_first[s] = (e >= 0 && first == s);
     }
-    u.start[n] = m;
-    u.n = n;
+    __syncthreads();
+    if (s < TK && e >= 0 && first == s) {   // rank among the distinct experts
+        int rank = 0;
+        for (int q = 0; q < s; ++q) rank += is_first[q];
+        u.u_of[s] = rank;
+        u.expert[rank] = e;
+    }
+    __syncthreads();
+    if (s < TK && e >= 0 && first != s) u.u_of[s] = u.u_of[first];
+    __syncthreads();
+    if (s <= TK) {                            // start[v]: slots of earlier experts
+        int c = 0;
+        for (int q = 0; q < TK; ++q) c += (u.e_of[q] >= 0 && u.u_of[q] < s);
+        u.start[s] = c;
+        if (s == 0) {
+            int n = 0;
+            for (int q = 0; q < TK; ++q) n += is_first[q];
+            u.n = n;
+        }
+    }
+    __syncthreads();
+    if (s < TK && e >= 0) {
+        int pos = u.start[u.u_of[s]];
+        for (int q = 0; q < s; ++q) pos += (u.e_of[q] == e);
+        u.slot[pos] = s;
+    }
+    __syncthreads();
 }
 
 __device__ __forceinline__ float dot8_bf16(const uint4 a, const uint4 b, float acc) {
@@ -78,73 +110,91 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
     return r;
 }
 
-// D1.  One item = (touched expert, feature); items split evenly over blocks.
-__global__ void __launch_bounds__(kUpWarps * 32) decode_up_bf16(
+// D1.  One item = (touched expert, feature f): gate row f and up row f are
+// loaded whole (VPL 16-byte vectors per lane each) before any use, and the
+// next item's rows are requested before the current one is reduced, so every
+// warp keeps up to 4*VPL*512 bytes in flight.  Items are split evenly over
+// blocks.
+template <int VPL>
+struct UpRows {
+    uint4 g[VPL], u[VPL];
+};
+
+template <int VPL>
+__device__ __forceinline__ void up_load(UpRows<VPL> &r, const uint4 *__restrict__ gate_up,
+                                        const Touched &tu, int64_t it, int F, int nv, int lane) {
+    const int ui = (int)(it / F), f = (int)(it - (int64_t)ui * F);
+    const uint4 *grow = gate_up + ((int64_t)tu.expert[ui] * 2 * F + f) * nv;
+    const uint4 *urow = grow + (int64_t)F * nv;
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+        const int v = c * 32 + lane;
+        r.g[c] = v < nv ? ld_stream(grow + v) : make_uint4(0, 0, 0, 0);
+        r.u[c] = v < nv ? ld_stream(urow + v) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+template <int VPL>
+__device__ __forceinline__ void up_compute(const UpRows<VPL> &r, const uint4 *__restrict__ x,
+                                           const Touched &tu, int64_t it, int F, int K, int nv,
+                                           int lane, __nv_bfloat16 *__restrict__ h) {
+    const int ui = (int)(it / F), f = (int)(it - (int64_t)ui * F);
+    for (int q = tu.start[ui]; q < tu.start[ui + 1]; ++q) {
+        const int slot = tu.slot[q];
+        const uint4 *xr = x + (int64_t)(slot / K) * nv;
+        float ga = 0.f, ua = 0.f;
+#pragma unroll
+        for (int c = 0; c < VPL; ++c) {
+            const int v = c * 32 + lane;
+            if (v < nv) {
+                const uint4 xv = __ldg(xr + v);
+                ga = dot8_bf16(r.g[c], xv, ga);
+                ua = dot8_bf16(r.u[c], xv, ua);
+            }
+        }
+        const float g = warp_sum(ga);
+        const float u = warp_sum(ua);
+        if (lane == 0) h[(int64_t)slot * F + f] = __float2bfloat16_rn(silu_f(g) * u);
+    }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(kUpWarps * 32, 1) decode_up_bf16(
     const uint4 *__restrict__ x, const uint4 *__restrict__ gate_up, const int32_t *__restrict__ idx,
     int T, int H, int F, int E, int K, __nv_bfloat16 *__restrict__ h) {
     __shared__ Touched tu;
-    if (threadIdx.x == 0) build_touched(idx, T * K, E, tu);
-    __syncthreads();
+    build_touched(idx, T * K, E, tu);
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int nv = H / 8;
     const int64_t items = (int64_t)tu.n * F;
     const int64_t i0 = items * blockIdx.x / gridDim.x, i1 = items * (blockIdx.x + 1) / gridDim.x;
-    for (int64_t it = i0 + warp; it < i1; it += kUpWarps) {
-        const int ui = (int)(it / F), f = (int)(it - (int64_t)ui * F);
-        const int e = tu.expert[ui];
-        const uint4 *grow = gate_up + ((int64_t)e * 2 * F + f) * nv;
-        const uint4 *urow = grow + (int64_t)F * nv;
-        for (int g0 = tu.start[ui]; g0 < tu.start[ui + 1]; g0 += kSlotGroup) {
-            const int ns = min(kSlotGroup, tu.start[ui + 1] - g0);
-            float ga[kSlotGroup] = {}, ua[kSlotGroup] = {};
-            for (int v0 = 0; v0 < nv; v0 += 32 * kChunkVec) {
-                uint4 wg[kChunkVec], wu[kChunkVec];
-#pragma unroll
-                for (int c = 0; c < kChunkVec; ++c) {
-                    const int v = v0 + c * 32 + lane;
-                    wg[c] = v < nv ? ld_stream(grow + v) : make_uint4(0, 0, 0, 0);
-                    wu[c] = v < nv ? ld_stream(urow + v) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int si = 0; si < kSlotGroup; ++si) {
-                    if (si < ns) {
-                        const uint4 *xr = x + (int64_t)(tu.slot[g0 + si] / K) * nv;
-#pragma unroll
-                        for (int c = 0; c < kChunkVec; ++c) {
-                            const int v = v0 + c * 32 + lane;
-                            if (v < nv) {
-                                const uint4 xv = __ldg(xr + v);
-                                ga[si] = dot8_bf16(wg[c], xv, ga[si]);
-                                ua[si] = dot8_bf16(wu[c], xv, ua[si]);
-                            }
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int si = 0; si < kSlotGroup; ++si) {
-                if (si < ns) {
-                    const float g = warp_sum(ga[si]);
-                    const float u = warp_sum(ua[si]);
-                    if (lane == 0)
-                        h[(int64_t)tu.slot[g0 + si] * F + f] = __float2bfloat16_rn(silu_f(g) * u);
-                }
-            }
-        }
+    UpRows<VPL> ra, rb;
+    int64_t it = i0 + warp;
+    if (it < i1) up_load(ra, gate_up, tu, it, F, nv, lane);
+    for (; it < i1; it += 2 * kUpWarps) {
+        const int64_t nb = it + kUpWarps, na = it + 2 * kUpWarps;
+        if (nb < i1) up_load(rb, gate_up, tu, nb, F, nv, lane);
+        up_compute(ra, x, tu, it, F, K, nv, lane, h);
+        if (na < i1) up_load(ra, gate_up, tu, na, F, nv, lane);
+        if (nb < i1) up_compute(rb, x, tu, nb, F, K, nv, lane, h);
     }
 }
 
-// D2.  One item = hidden row j; rows split evenly over blocks.
-__global__ void __launch_bounds__(kDownWarps * 32) decode_down_bf16(
+// D2.  Block b owns hidden rows [j0, j1).  One item = (row j, touched expert
+// u); a warp loads the down rows of two items before using either.  The
+// per-slot results y_s land in shared memory; after a block barrier,
+// out[t, j] = bf16( sum_{k in order} w[t,k] * y_{t*K+k} ).
+template <int VPL>
+__global__ void __launch_bounds__(kDownWarps * 32, VPL <= 4 ? 2 : 1) decode_down_bf16(
     const uint4 *__restrict__ down, const uint4 *__restrict__ h, const int32_t *__restrict__ idx,
     const float *__restrict__ w, int T, int H, int F, int E, int K, __nv_bfloat16 *__restrict__ out) {
     __shared__ Touched tu;
-    __shared__ float ys[kDownWarps][kDecodeMaxSlots];
-    if (threadIdx.x == 0) build_touched(idx, T * K, E, tu);
-    __syncthreads();
+    extern __shared__ float ys[];     // [rows of this block][T*K]
+    build_touched(idx, T * K, E, tu);
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int nv = F / 8;
+    const int TK = T * K;
     const int j0 = (int)((int64_t)H * blockIdx.x / gridDim.x);
     const int j1 = (int)((int64_t)H * (blockIdx.x + 1) / gridDim.x);
     // Stream this block's down rows into L2 while D1 is still running.
@@ -152,28 +202,36 @@ __global__ void __launch_bounds__(kDownWarps * 32) decode_down_bf16(
         prefetch_l2_bulk(down + ((int64_t)tu.expert[threadIdx.x] * H + j0) * nv,
                          (uint32_t)((j1 - j0) * F * 2));
     pdl_wait();
-    for (int j = j0 + warp; j < j1; j += kDownWarps) {
-        for (int ui = 0; ui < tu.n; ++ui) {
-            const uint4 *drow = down + ((int64_t)tu.expert[ui] * H + j) * nv;
+    const int items = (j1 - j0) * tu.n;
+    for (int i = 2 * warp; i < items; i += 2 * kDownWarps) {
+        uint4 wd[2][VPL];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int it = i + p;
+            const int jl = it / max(tu.n, 1), ui = it - jl * tu.n;
+            const uint4 *drow = down + ((int64_t)tu.expert[it < items ? ui : 0] * H + j0 + jl) * nv;
+#pragma unroll
+            for (int c = 0; c < VPL; ++c) {
+                const int v = c * 32 + lane;
+                wd[p][c] = (it < items && v < nv) ? __ldg(drow + v) : make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const int it = i + p;
+            if (it >= items) break;
+            const int jl = it / tu.n, ui = it - jl * tu.n;
             for (int g0 = tu.start[ui]; g0 < tu.start[ui + 1]; g0 += kSlotGroup) {
                 const int ns = min(kSlotGroup, tu.start[ui + 1] - g0);
                 float ya[kSlotGroup] = {};
-                for (int v0 = 0; v0 < nv; v0 += 32 * kChunkVec) {
-                    uint4 wd[kChunkVec];
 #pragma unroll
-                    for (int c = 0; c < kChunkVec; ++c) {
-                        const int v = v0 + c * 32 + lane;
-                        wd[c] = v < nv ? __ldg(drow + v) : make_uint4(0, 0, 0, 0);
-                    }
+                for (int si = 0; si < kSlotGroup; ++si) {
+                    if (si < ns) {
+                        const uint4 *hr = h + (int64_t)tu.slot[g0 + si] * nv;
 #pragma unroll
-                    for (int si = 0; si < kSlotGroup; ++si) {
-                        if (si < ns) {
-                            const uint4 *hr = h + (int64_t)tu.slot[g0 + si] * nv;
-#pragma unroll
-                            for (int c = 0; c < kChunkVec; ++c) {
-                                const int v = v0 + c * 32 + lane;
-                                if (v < nv) ya[si] = dot8_bf16(wd[c], __ldg(hr + v), ya[si]);
-                            }
+                        for (int c = 0; c < VPL; ++c) {
+                            const int v = c * 32 + lane;
+                            if (v < nv) ya[si] = dot8_bf16(wd[p][c], __ldg(hr + v), ya[si]);
                         }
                     }
                 }
@@ -181,23 +239,22 @@ __global__ void __launch_bounds__(kDownWarps * 32) decode_down_bf16(
                 for (int si = 0; si < kSlotGroup; ++si) {
                     if (si < ns) {
                         const float y = warp_sum(ya[si]);
-                        if (lane == 0) ys[warp][tu.slot[g0 + si]] = y;
+                        if (lane == 0) ys[jl * TK + tu.slot[g0 + si]] = y;
                     }
                 }
             }
         }
-        __syncwarp();
-        if (lane < T) {
-            float acc = 0.f;
-            for (int k = 0; k < K; ++k) {
-                const int s = lane * K + k;
-                const int e = idx[s];
-                if (e < 0 || e >= E) continue;
-                acc = fmaf(w[s], ys[warp][s], acc);
-            }
-            out[(int64_t)lane * H + j] = __float2bfloat16_rn(acc);
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < (j1 - j0) * T; q += blockDim.x) {
+        const int jl = q / T, t = q - jl * T;
+        float acc = 0.f;
+        for (int k = 0; k < K; ++k) {
+            const int s = t * K + k;
+            if (tu.e_of[s] < 0) continue;
+            acc = fmaf(w[s], ys[jl * TK + s], acc);
         }
-        __syncwarp();
+        out[(int64_t)t * H + j0 + jl] = __float2bfloat16_rn(acc);
     }
 }
 
@@ -207,14 +264,43 @@ cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *d
                                const int32_t *idx, const float *w, int T, int H, int F, int E,
                                int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
                                cudaStream_t st) {
-    const int sms = num_sms();
     __nv_bfloat16 *h = (__nv_bfloat16 *)(ws + L.h);
-    cudaError_t err = launch_k(decode_up_bf16, dim3(sms), dim3(kUpWarps * 32), 0, st, false,
-                               (const uint4 *)x, (const uint4 *)gate_up, idx, T, H, F, E, K, h);
+    const int vpl_up = (H / 8 + 31) / 32, vpl_dn = (F / 8 + 31) / 32;
+    int grid = num_sms();
+    const dim3 blk(kUpWarps * 32);
+    cudaError_t err;
+#define MOE_UP(V) launch_k(decode_up_bf16<V>, dim3(grid), blk, 0, st, false, (const uint4 *)x, \
+                           (const uint4 *)gate_up, idx, T, H, F, E, K, h)
+    switch (vpl_up) {
+        case 1: err = MOE_UP(1); break;
+        case 2: err = MOE_UP(2); break;
+        case 3: err = MOE_UP(3); break;
+        case 4: err = MOE_UP(4); break;
+        case 5: err = MOE_UP(5); break;
+        case 6: err = MOE_UP(6); break;
+        case 7: err = MOE_UP(7); break;
+        case 8: err = MOE_UP(8); break;
+        default: return cudaErrorInvalidValue;
+    }
+#undef MOE_UP
     if (err != cudaSuccess) return err;
-    return launch_k(decode_down_bf16, dim3(sms), dim3(kDownWarps * 32), 0, st, true,
-                    (const uint4 *)down, (const uint4 *)h, idx, w, T, H, F, E, K,
-                    (__nv_bfloat16 *)out);
+    grid = (vpl_dn <= 4 ? 2 : 1) * num_sms();
+    const size_t smem = sizeof(float) * ((H + grid - 1) / grid + 1) * T * K;
+#define MOE_DN(V) launch_k(decode_down_bf16<V>, dim3(grid), dim3(kDownWarps * 32), smem, st, true, \
+                           (const uint4 *)down, (const uint4 *)h, idx, w, T, H, F, E, K,        \
+                           (__nv_bfloat16 *)out)
+    switch (vpl_dn) {
+        case 1: return MOE_DN(1);
+        case 2: return MOE_DN(2);
+        case 3: return MOE_DN(3);
+        case 4: return MOE_DN(4);
+        case 5: return MOE_DN(5);
+        case 6: return MOE_DN(6);
+        case 7: return MOE_DN(7);
+        case 8: return MOE_DN(8);
+        default: return cudaErrorInvalidValue;
+    }
+#undef MOE_DN
 }
 
 }  // namespace moe

@@ -17,7 +17,8 @@
 // the device; the host never synchronises).  Warp roles:
 //   warp 0     TMA producer (4-stage shared-memory ring)
 //   warp 1     TMEM allocation + MMA issue (one thread)
-//   warps 2-5  epilogue: TMEM -> registers -> global (double-buffered TMEM)
+//   warps 2-9  epilogue: TMEM -> registers -> global (double-buffered TMEM);
+//              two warps per TMEM lane quarter, alternating 32-column chunks
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -30,7 +31,8 @@ namespace {
 constexpr int kStages = 4;
 constexpr int kBK = 64;           // bf16 elements per k-block = one 128-byte swizzle row
 constexpr int kBoxRows = 32;      // routed rows per TMA box of the B operand
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 template <bool GATE_UP>
 struct Cfg {
@@ -42,7 +44,10 @@ struct Cfg {
     static constexpr int ACC_COLS = NUM_A * BN;        // TMEM columns per accumulator set
     static constexpr int NUM_ACC = 512 / ACC_COLS;     // accumulator sets (2)
     static constexpr int RING_BYTES = kStages * STAGE_BYTES;
-    static size_t smem_bytes(int E) { return RING_BYTES + 1024 + 1024 + 2 * sizeof(int) * (E + 1); }
+    static constexpr int STAGE_OUT = kEpiWarps * 32 * 32 * 2;   // h staging, 2 KB per warp
+    static size_t smem_bytes(int E) {
+        return RING_BYTES + 1024 + 1024 + STAGE_OUT + align_up(2 * sizeof(int) * (E + 1), 16);
+    }
 };
 
 struct GemmArgs {
@@ -64,6 +69,9 @@ struct Tile {
     int e, m, row0, nrows;
 };
 
+// Work item w -> (expert, weight-row tile, routed rows).  Items of one expert
+// are contiguous, routed-row tiles fastest; an expert's n_e rows are split in
+// ceil(n_e/BN) near-equal tiles of a multiple of 16 rows.
 __device__ __forceinline__ Tile decode_tile(int w, const int32_t *s_off, const int32_t *s_tiles,
                                             int E, int MT, int BN) {
     int lo = 0, hi = E;  // s_tiles[lo]*MT <= w < s_tiles[hi]*MT
@@ -77,8 +85,10 @@ __device__ __forceinline__ Tile decode_tile(int w, const int32_t *s_off, const i
     const int local = w - s_tiles[lo] * MT;
     t.m = local / nt;
     const int n = local - t.m * nt;
-    t.row0 = s_off[lo] + n * BN;
-    t.nrows = min(BN, s_off[lo + 1] - t.row0);
+    const int n_e = s_off[lo + 1] - s_off[lo];
+    const int rpt = min(BN, ((n_e + nt - 1) / nt + 15) & ~15);
+    t.row0 = s_off[lo] + n * rpt;
+    t.nrows = min(rpt, n_e - n * rpt);
     return t;
 }
 
@@ -97,7 +107,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *tempty = tfull + C::NUM_ACC;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + C::NUM_ACC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int32_t *s_off = reinterpret_cast<int32_t *>(smem + C::RING_BYTES + 1024);
+    __nv_bfloat16 *s_out = reinterpret_cast<__nv_bfloat16 *>(smem + C::RING_BYTES + 1024);
+    int32_t *s_off = reinterpret_cast<int32_t *>(smem + C::RING_BYTES + 1024 + C::STAGE_OUT);
     int32_t *s_tiles = s_off + (args.E + 1);
 
     const int warp = threadIdx.x >> 5, lane = lane_id();
@@ -108,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int a = 0; a < C::NUM_ACC; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 32 * kEpiWarps);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -215,8 +226,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue --------
+        const int ew = warp - 2;                // 0 .. kEpiWarps-1
         const int eg = warp & 3;                // TMEM lanes [32*eg, 32*eg+32)
+        const int half = ew >> 2;               // which 32-column chunks
         const int row = eg * 32 + lane;         // weight row inside the tile
+        __nv_bfloat16 *stg = s_out + ew * 32 * 32;   // [32 rows][32 features]
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -228,21 +242,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + acc * C::ACC_COLS;
-            for (int c0 = 0; c0 < t.nrows; c0 += 32) {
+            for (int c0 = half * 32; c0 < t.nrows; c0 += 64) {
                 uint32_t g[32];
                 tmem_ld32(tb + c0, g);
                 if (GATE_UP) {
                     uint32_t u[32];
                     tmem_ld32(tb + C::BN + c0, u);
                     tmem_ld_wait();
-                    __nv_bfloat16 *hp = args.h + (size_t)(t.row0 + c0) * args.F + t.m * kBM + row;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        if (c0 + j < t.nrows) {
-                            const float gv = __uint_as_float(g[j]);
-                            hp[(size_t)j * args.F] = __float2bfloat16_rn(silu_f(gv) * __uint_as_float(u[j]));
+                        const float gv = __uint_as_float(g[j]);
+                        const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(u[j]);
+                        stg[j * 32 + lane] = __float2bfloat16_rn(hv);
+                    }
+                    __syncwarp();
+                    // 32 routed rows x 64 bytes: four lanes per row, 16 bytes each
+                    const int q = lane & 3;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = (lane >> 2) + 8 * i;
+                        if (c0 + r < t.nrows) {
+                            const uint4 v = *reinterpret_cast<const uint4 *>(stg + r * 32 + q * 8);
+                            *reinterpret_cast<uint4 *>(args.h + (size_t)(t.row0 + c0 + r) * args.F +
+                                                       t.m * kBM + eg * 32 + q * 8) = v;
                         }
                     }
+                    __syncwarp();
                 } else {
                     tmem_ld_wait();
                     const int c = c0 + lane;

@@ -140,6 +140,90 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t *__restrict__ chunk_
     pdl_launch_dependents();
 }
 
+// Whole permutation in one block of 1024 threads, for up to
+// kSmallSlots slots: warp w takes slots [w*R, (w+1)*R), R = 32*rounds, and
+// ranks them as hist_kernel does; then per-expert bases over the warps,
+// expert counts / offsets / tile prefixes, and the final positions.
+// smem: 32 x E counters + E+1 offsets.
+constexpr int kSmallRounds = 16;
+constexpr int kSmallSlots = 1024 * kSmallRounds;
+
+__global__ void __launch_bounds__(1024) permute_small_kernel(
+    const int32_t *__restrict__ idx, int n_slots, int E, int32_t *__restrict__ counts,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ tiles_g, int32_t *__restrict__ tiles_d,
+    int32_t *__restrict__ perm, int32_t *__restrict__ inv, int32_t *__restrict__ status) {
+    extern __shared__ int32_t sm[];
+    int32_t *wcnt = sm;                 // [32][E]
+    int32_t *s_off = sm + 32 * E;       // [E+1]
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    if (threadIdx.x == 0) *status = 0;
+    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+    const int rounds = (n_slots + 1023) / 1024;
+    const int base = warp * rounds * 32;
+    int loc[kSmallRounds], ex[kSmallRounds];
+#pragma unroll
+    for (int r = 0; r < kSmallRounds; ++r) {
+        ex[r] = -1;
+        const int s = base + r * 32 + lane;
+        if (r < rounds && s < n_slots) {
+            const int e = __ldg(idx + s);
+            if (e >= 0 && e < E) ex[r] = e;
+        }
+    }
+    __syncthreads();
+    const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (int r = 0; r < kSmallRounds; ++r) {
+        if (r < rounds) {
+            const int e = ex[r];
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+            const int rank = __popc(peers & lt_mask);
+            const int prior = (e >= 0) ? wcnt[warp * E + e] : 0;
+            __syncwarp();
+            if (e >= 0 && rank == 0) wcnt[warp * E + e] = prior + __popc(peers);
+            __syncwarp();
+            loc[r] = prior + rank;
+        }
+    }
+    __syncthreads();
+    int n = 0;
+    const int e = threadIdx.x;
+    if (e < E) {
+        for (int w = 0; w < 32; ++w) {
+            const int v = wcnt[w * E + e];
+            wcnt[w * E + e] = n;
+            n += v;
+        }
+        counts[e] = n;
+    }
+    int total = 0;
+    const int off = block_exclusive_scan(n, total);
+    if (e < E) { offsets[e] = off; s_off[e] = off; }
+    if (e == 0) { offsets[E] = total; s_off[E] = total; }
+    const int tgo = block_exclusive_scan((n + kBNGateUp - 1) / kBNGateUp, total);
+    if (e < E) tiles_g[e] = tgo;
+    if (e == 0) tiles_g[E] = total;
+    const int tdo = block_exclusive_scan((n + kBNDown - 1) / kBNDown, total);
+    if (e < E) tiles_d[e] = tdo;
+    if (e == 0) tiles_d[E] = total;
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kSmallRounds; ++r) {
+        const int s = base + r * 32 + lane;
+        if (r < rounds && s < n_slots) {
+            if (ex[r] >= 0) {
+                const int pos = s_off[ex[r]] + wcnt[warp * E + ex[r]] + loc[r];
+                perm[pos] = s;
+                inv[s] = pos;
+            } else {
+                inv[s] = -1;
+            }
+        }
+    }
+    for (int p = s_off[E] + threadIdx.x; p < n_slots; p += blockDim.x) perm[p] = -1;
+    pdl_launch_dependents();
+}
+
 // Final slot positions.  One thread per slot; also fills perm entries past
 // offsets[E] (slots whose expert id is out of range) with -1.
 __global__ void __launch_bounds__(256) scatter_kernel(
@@ -238,6 +322,24 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
 
 cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, uint8_t *ws,
                            const Workspace &L, cudaStream_t st) {
+    if (n_slots <= kSmallSlots) {
+        const size_t smem = sizeof(int32_t) * (33 * (size_t)E + 1);
+        static int attr_done[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (!attr_done[dev & 63]) {
+            cudaError_t e = cudaFuncSetAttribute(permute_small_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)(sizeof(int32_t) * (33 * 1024 + 1)));
+            if (e != cudaSuccess) return e;
+            attr_done[dev & 63] = 1;
+        }
+        return launch_k(permute_small_kernel, dim3(1), dim3(1024), smem, st, false, idx,
+                        (int)n_slots, E, (int32_t *)(ws + L.counts), (int32_t *)(ws + L.offsets),
+                        (int32_t *)(ws + L.tiles_g), (int32_t *)(ws + L.tiles_d),
+                        (int32_t *)(ws + L.perm), (int32_t *)(ws + L.inv),
+                        (int32_t *)(ws + L.status));
+    }
     const int n_chunks = (int)((n_slots + kChunk - 1) / kChunk);
     int32_t *status = (int32_t *)(ws + L.status);
     int32_t *chunk_hist = (int32_t *)(ws + L.chunk_hist);
