@@ -130,6 +130,33 @@ MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *g
                                 size_t workspace_bytes, void *stream);
 
 /*
+ * Decode form without a workspace, for callers that cannot allocate device
+ * memory where they run the layer: code recorded into a CUDA graph while
+ * capture forbids allocation, serving loops and real-time hosts that fix
+ * their device memory budget at start-up, plugin or embedded hosts that give
+ * the code they load no allocator.  The pages have no counterpart of this
+ * entry point; it exists for those callers only.
+ *
+ * Same arguments, layouts and results as moe_experts_decode, minus the
+ * workspace.  Its scratch memory is a fixed 1 MiB array inside the library
+ * that every GPU which loads the library holds until the process exits.
+ * The library itself allocates nothing and calls no allocating routine.
+ *  - Sizes whose decode scratch (moe_experts_workspace_size(..., 1)) exceeds
+ *    1 MiB, and calls outside the decode range (T > 16 or T*K > 64), return
+ *    MOE_ERR_WORKSPACE; e4m3 weights return MOE_ERR_UNSUPPORTED.
+ *  - The first call on a device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents:
+ *    calls that may overlap on the GPU (other streams, or other host threads
+ *    without ordering) race on it and must be serialised by the caller.
+ */
+MOE_API moe_status_t moe_experts_decode_static(const void *hidden_states, const void *gate_up_proj,
+                                       const void *down_proj, const int32_t *top_k_index,
+                                       const float *top_k_weights, int top_k, int T, int H, int F,
+                                       int E, moe_wtype_t wt, const float *gate_up_scale,
+                                       const float *down_scale, void *out, void *stream);
+
+/*
  * Group-aware sigmoid top-k routing (layer table:
  * moe_topk_sigmoid_routing_layer, num_groups=8, topk_group=4,
  * routed_scaling_factor=2.5 for DeepSeek-V3).

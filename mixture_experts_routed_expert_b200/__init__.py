@@ -24,7 +24,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 
 EXPORTS = ("moe_abi_version", "moe_status_string", "moe_experts_workspace_size",
            "moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
-           "quantize_fp8_block128", "moe_debug_permute")
+           "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static")
 
 
 def _load():
@@ -45,7 +45,7 @@ def _load():
     L.quantize_fp8_block128.argtypes = [P, I, I, P, P, P]
     L.moe_debug_permute.argtypes = [P, I, I, I, P, P, P, P, P, Z, P]
     for n in ("moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
-              "quantize_fp8_block128", "moe_debug_permute"):
+              "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static"):
         getattr(L, n).restype = I
     return L
 
@@ -128,6 +128,23 @@ def moe_experts_decode(hidden_states, gate_up_proj, down_proj, top_k_index, top_
     """Routed-experts forward, fused gather-GEMV form for a few tokens."""
     return _forward("moe_experts_decode", hidden_states, gate_up_proj, down_proj, top_k_index,
                     top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream)
+
+
+def moe_experts_decode_static(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
+                              top_k, gate_up_scale=None, down_scale=None, out=None, stream=None):
+    """Decode form without a workspace: scratch comes from a fixed 1 MiB array
+    inside the library (for callers that cannot allocate device memory; calls
+    that overlap on the GPU race on that array)."""
+    T, H = hidden_states.shape
+    E, F2, _ = gate_up_proj.shape
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
+    rc = lib.moe_experts_decode_static(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
+                                       _ptr(top_k_index), _ptr(top_k_weights), top_k, T, H, F2 // 2,
+                                       E, _wtype(gate_up_proj), _ptr(gate_up_scale),
+                                       _ptr(down_scale), _ptr(out), _stream(stream))
+    _check(rc, "moe_experts_decode_static")
+    return out
 
 
 def moe_route_sigmoid_grouped(logits, bias, num_groups, topk_group, top_k, routed_scaling_factor,

@@ -132,6 +132,16 @@ moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const in
 
 }  // namespace
 
+namespace moe {
+// Validation and decode-size rule shared with the other entry points.
+moe_status_t validate_forward(const void *x, const void *gu, const void *dn, const int32_t *idx,
+                              const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
+                              const float *gus, const float *dns, const void *out) {
+    return check_common(x, gu, dn, idx, w, K, T, H, F, E, wt, gus, dns, out);
+}
+bool decode_path_fits(int T, int K) { return decode_fits(T, K); }
+}  // namespace moe
+
 extern "C" {
 
 int moe_abi_version(void) { return 1; }

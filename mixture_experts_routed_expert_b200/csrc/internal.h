@@ -49,6 +49,13 @@ DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t 
 constexpr int kDecodeMaxSlots = 64;  // T*K served by the decode kernels
 constexpr int kDecodeMaxT = 16;
 
+// Host-side argument checks of the forward entry points (MOE_OK when valid).
+moe_status_t validate_forward(const void *x, const void *gu, const void *dn, const int32_t *idx,
+                              const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
+                              const float *gus, const float *dns, const void *out);
+// True when T tokens x K slots are served by the decode kernels.
+bool decode_path_fits(int T, int K);
+
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 int num_sms();
 
