@@ -6,8 +6,10 @@
 One step = one routed-experts MoE layer on the OCR-2 decode shape
 (T=1 token, H=1280, F=896, E=64 experts, top-6, bf16; synthetic seeded
 inputs, all 64 experts' weights resident in HBM), run through the C ABI of
-libmoe_b200.so and replayed from a CUDA graph.  L2 is flushed (a 512 MiB
-buffer is written) before every timed step, outside the timed interval.
+libmoe_b200.so and replayed from a CUDA graph.  L2 is flushed before every
+timed step, outside the timed interval: a 512 MiB buffer is written, then a
+separate 256 MiB buffer is read, so the step starts with none of its own data
+in L2 and without dirty lines left behind by the flush.
 Each step is timed with CUDA events on the launching stream; the JSON line
 reports the sum over the K timed steps, max over ranks.
 
@@ -42,6 +44,7 @@ sys.path.insert(0, ROOT)
 PAGES_DECODE_T1_US = 191.0       # model card, GB10 decode latency (context only)
 METRIC = "us_per_moe_layer"
 FLUSH_BYTES = 512 << 20
+FLUSH_READ_BYTES = 256 << 20
 
 
 def load_peaks():
@@ -133,7 +136,12 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     peaks = load_peaks()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def flush(i):
+        flush_w.fill_(i & 0xFF)
+        flush_r.sum()
 
     def barrier():
         if world > 1:
@@ -157,7 +165,7 @@ def run_ours(args):
         with torch.cuda.graph(g):
             fn()
         for _ in range(warmup):
-            flush.fill_(1)
+            flush(1)
             g.replay()
         torch.cuda.synchronize()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -165,7 +173,7 @@ def run_ours(args):
         barrier()
         torch.cuda.synchronize()
         for i in range(steps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             evs[i][0].record(stream)
             g.replay()
             evs[i][1].record(stream)
@@ -175,13 +183,13 @@ def run_ours(args):
 
     def time_eager(fn, steps, warmup):
         for _ in range(warmup):
-            flush.fill_(1)
+            flush(1)
             fn()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(steps)]
         torch.cuda.synchronize()
         for i in range(steps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             evs[i][0].record(stream)
             fn()
             evs[i][1].record(stream)
@@ -271,7 +279,7 @@ def run_ours(args):
         "dtype": "bf16", "data": "synthetic (seeded N(0,1) hidden, N(0,0.02^2) weights, softmax top-6 routing)",
         "config": {"workload": "OCR-2 routed experts, decode T=1 (H=1280 F=896 E=64 K=6, bf16)",
                    "global_batch": world, "seq_len": 1, "parallelism": "replicas%d" % world,
-                   "l2": "flushed (512 MiB write) before every timed step",
+                   "l2": "flushed before every timed step (512 MiB write, then 256 MiB read)",
                    "timing": "CUDA graph replay of the C-ABI call, CUDA events"},
         "roofline": {"bound": "hbm", "kernel": "decode_up_bf16 + decode_down_bf16 (PDL chain)",
                      "achieved": round(achieved, 1), "peak": peaks["hbm"], "unit": "GB/s",
@@ -305,10 +313,12 @@ def run_only(args):
     T = {"decode1": 1, "decode4": 4, "prefill2048": 2048}[args.only]
     fn = moe.moe_experts_prefill if args.only.startswith("prefill") else moe.moe_experts_decode
     lay = inputs.ocr2_layer(T, seed=T, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
     out = None
     for i in range(args.warmup + args.steps):
-        flush.fill_(i & 0xFF)
+        flush_w.fill_(i & 0xFF)
+        flush_r.sum()
         out = fn(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, 6)
     torch.cuda.synchronize()
     print("ok", args.only, float(out.float().abs().sum()))

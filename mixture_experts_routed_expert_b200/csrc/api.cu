@@ -75,13 +75,13 @@ Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t w
 }
 
 DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t wt) {
-    (void)H;
     (void)E;
     const size_t N = (size_t)T * K;
     DecodeWorkspace L;
     Bump b;
-    L.status = b.take(16);
+    L.sync = b.take(sizeof(int32_t) * decode_sync_ints(H));
     L.h = b.take(2 * N * F);
+    L.ys = b.take(0);
     L.hq = b.take(wt == MOE_W_BF16 ? 0 : N * F);
     L.hscale = b.take(wt == MOE_W_BF16 ? 0 : sizeof(float) * N * (F / 128));
     L.total = b.off;
@@ -94,7 +94,9 @@ using namespace moe;
 
 namespace {
 
-bool decode_fits(int T, int K) { return T <= kDecodeMaxT && T * K <= kDecodeMaxSlots; }
+bool decode_fits(int T, int K, int H, int F) {
+    return T <= kDecodeMaxT && T * K <= kDecodeMaxSlots && decode_shape_ok(H, F);
+}
 
 moe_status_t check_common(const void *x, const void *gu, const void *dn, const int32_t *idx,
                           const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
@@ -139,7 +141,7 @@ moe_status_t validate_forward(const void *x, const void *gu, const void *dn, con
                               const float *gus, const float *dns, const void *out) {
     return check_common(x, gu, dn, idx, w, K, T, H, F, E, wt, gus, dns, out);
 }
-bool decode_path_fits(int T, int K) { return decode_fits(T, K); }
+bool decode_path_fits(int T, int K, int H, int F) { return decode_fits(T, K, H, F); }
 }  // namespace moe
 
 extern "C" {
@@ -160,7 +162,7 @@ const char *moe_status_string(moe_status_t s) {
 
 size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t wt, int decode) {
     if (!dims_ok(T, H, F, E, K)) return 0;
-    if (decode && decode_fits(T, K)) return decode_workspace(T, H, F, E, K, wt).total;
+    if (decode && decode_fits(T, K, H, F)) return decode_workspace(T, H, F, E, K, wt).total;
     return prefill_workspace(T, H, F, E, K, wt).total;
 }
 
@@ -190,7 +192,7 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
                                   out);
     if (s != MOE_OK || T == 0) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    if (!decode_fits(T, top_k))
+    if (!decode_fits(T, top_k, H, F))
         return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                            top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
                            workspace_bytes, st);

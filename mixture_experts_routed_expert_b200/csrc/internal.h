@@ -38,12 +38,17 @@ struct Workspace {
 Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t wt);
 
 struct DecodeWorkspace {
-    size_t status;
+    size_t sync;          // int32: status word (+3 spare)
     size_t h;             // [T*K][F] bf16
-    size_t hq;            // [T*K][F] e4m3 + scales (e4m3 path)
-    size_t hscale;
+    size_t ys;            // unused (kept empty)
+    size_t hq;            // [T*K][F] e4m3 (e4m3 path)
+    size_t hscale;        // [T*K][F/128] f32 (e4m3 path)
     size_t total;
 };
+// int32 entries of the decode sync region for hidden size H.
+size_t decode_sync_ints(int H);
+// True when the decode kernel's shared-memory staging fits these sizes.
+bool decode_shape_ok(int H, int F);
 DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t wt);
 
 constexpr int kDecodeMaxSlots = 64;  // T*K served by the decode kernels
@@ -54,7 +59,7 @@ moe_status_t validate_forward(const void *x, const void *gu, const void *dn, con
                               const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
                               const float *gus, const float *dns, const void *out);
 // True when T tokens x K slots are served by the decode kernels.
-bool decode_path_fits(int T, int K);
+bool decode_path_fits(int T, int K, int H, int F);
 
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 int num_sms();

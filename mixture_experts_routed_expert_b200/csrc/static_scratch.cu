@@ -65,7 +65,7 @@ extern "C" MOE_API moe_status_t moe_experts_decode_static(
                                       top_k_weights, top_k, T, H, F, E, wt, gate_up_scale,
                                       down_scale, out);
     if (s != MOE_OK || T == 0) return s;
-    if (!decode_path_fits(T, top_k)) return MOE_ERR_WORKSPACE;
+    if (!decode_path_fits(T, top_k, H, F)) return MOE_ERR_WORKSPACE;
     if (wt != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
     const DecodeWorkspace L = decode_workspace(T, H, F, E, top_k, wt);
     if (L.total > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
