@@ -120,14 +120,15 @@ moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const in
                          cudaStream_t st) {
     const Workspace L = prefill_workspace(T, H, F, E, K, wt);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
-    if (wt != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
-    (void)gus;
-    (void)dns;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     const int64_t N = (int64_t)T * K;
-    cudaError_t e = launch_permute(idx, N, E, wsb, L, st);
+    const bool fp8 = (wt == MOE_W_FP8_E4M3);
+    cudaError_t e = fp8 ? launch_permute(idx, N, E, kBNFp8, kBNFp8, wsb, L, st)
+                        : launch_permute(idx, N, E, kBNGateUp, kBNDown, wsb, L, st);
     if (e == cudaSuccess) e = launch_gather(x, idx, N, K, H, E, wt, wsb, L, st);
-    if (e == cudaSuccess) e = launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st);
+    if (e == cudaSuccess)
+        e = fp8 ? launch_gemms_fp8(gu, gus, dn, dns, w, T, H, F, E, K, wsb, L, st)
+                : launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st);
     if (e == cudaSuccess) e = launch_combine(idx, T, H, E, K, wsb, L, out, st);
     return from_cuda(e);
 }
@@ -162,7 +163,8 @@ const char *moe_status_string(moe_status_t s) {
 
 size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t wt, int decode) {
     if (!dims_ok(T, H, F, E, K)) return 0;
-    if (decode && decode_fits(T, K, H, F)) return decode_workspace(T, H, F, E, K, wt).total;
+    if (decode && decode_fits(T, K, H, F) && wt == MOE_W_BF16)
+        return decode_workspace(T, H, F, E, K, wt).total;
     return prefill_workspace(T, H, F, E, K, wt).total;
 }
 
@@ -192,7 +194,7 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
                                   out);
     if (s != MOE_OK || T == 0) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    if (!decode_fits(T, top_k, H, F))
+    if (!decode_fits(T, top_k, H, F) || wt != MOE_W_BF16)
         return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                            top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
                            workspace_bytes, st);
@@ -251,7 +253,7 @@ moe_status_t moe_debug_permute(const int32_t *top_k_index, int T, int K, int E, 
         if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
         return from_cuda(e);
     }
-    cudaError_t e = launch_permute(top_k_index, N, E, ws, L, st);
+    cudaError_t e = launch_permute(top_k_index, N, E, kBNGateUp, kBNDown, ws, L, st);
     if (e == cudaSuccess) e = launch_debug_outputs(top_k_index, N, E, ws, L, counts, offsets, perm, inv, st);
     return from_cuda(e);
 }

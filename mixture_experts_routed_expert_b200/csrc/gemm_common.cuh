@@ -1,0 +1,67 @@
+// gemm_common.cuh -- pieces shared by the grouped GEMM kernels (bf16 and
+// E4M3): the tile list over experts and the TMA descriptor encoder.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+struct Tile {
+    int e, m, row0, nrows;
+};
+
+// Work item w -> (expert, weight-row tile, routed rows).  Items of one expert
+// are contiguous, routed-row tiles fastest; an expert's n_e rows are split in
+// ceil(n_e/BN) near-equal tiles of a multiple of 16 rows.
+__device__ __forceinline__ Tile decode_tile(int w, const int32_t *s_off, const int32_t *s_tiles,
+                                            int E, int MT, int BN) {
+    int lo = 0, hi = E;  // s_tiles[lo]*MT <= w < s_tiles[hi]*MT
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_tiles[mid] * MT <= w) lo = mid; else hi = mid;
+    }
+    Tile t;
+    t.e = lo;
+    const int nt = s_tiles[lo + 1] - s_tiles[lo];
+    const int local = w - s_tiles[lo] * MT;
+    t.m = local / nt;
+    const int n = local - t.m * nt;
+    const int n_e = s_off[lo + 1] - s_off[lo];
+    const int rpt = min(BN, ((n_e + nt - 1) / nt + 15) & ~15);
+    t.row0 = s_off[lo] + n * rpt;
+    t.nrows = min(rpt, n_e - n * rpt);
+    return t;
+}
+
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// Row-major [rows, cols] matrix, box = box_rows x 128 bytes, 128-byte swizzle.
+inline bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int elem_bytes, const void *ptr,
+               uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+
+}  // namespace moe

@@ -1,0 +1,375 @@
+// gemm_fp8.cu -- S4 and S5 of the prefill path for E4M3 expert weights with
+// fp32 scales per (row, 128-column block) and E4M3 activations with
+// power-of-two scales per 128 columns ("Supporting MegaKernel for DeepSeek
+// Models", layer table: moe_w13_fp8_layer, moe_silu_mul_layer,
+// bf16_to_fp8_quantize, moe_w2_fp8_layer).
+//
+// Grouped GEMM on tcgen05 with kind::f8f6f4 (E4M3 x E4M3 -> fp32, K = 32 per
+// instruction).  Because each 128-wide k-block has its own weight and
+// activation scale, every k-block's product goes to a TMEM "partial" buffer
+// (two, alternating); epilogue warps read it and promote it into fp32
+// accumulators held in registers:
+//     acc[row, col] += (w_scale[row, kb] * x_scale[col, kb]) * partial[row, col]
+// while the MMA of the next k-block fills the other partial buffer.
+//   S4 (gate_up):  tile = 128 features of expert e (gate rows and up rows,
+//     two partials) x up to 64 routed rows.  h = bf16(SiLU(g) * u), then
+//     quantised per 128 features (the tile's 128 rows): scale = smallest power
+//     of two with max|h|/scale <= 448, codes E4M3 -> hq [N][F], hs [N][F/128].
+//   S5 (down):  tile = 128 hidden rows x up to 64 routed rows;
+//     y[slot, j] = w[slot] * acc  (fp32, by original slot; combined later).
+// Warp roles as in the bf16 kernel: warp 0 TMA producer, warp 1 TMEM
+// allocation + MMA issue, warps 2-9 promotion and epilogue (two warps per TMEM
+// lane quarter, each owning 32 of the 64 columns).
+#include "common.cuh"
+#include "gemm_common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBN8 = kBNFp8;          // routed rows per tile
+constexpr int kEpi8 = 8;
+constexpr int kThreads8 = 64 + 32 * kEpi8;
+constexpr int kMaxKB8 = 128;          // k-blocks (of 128) per row supported
+
+template <bool GATE_UP>
+struct Cfg8 {
+    static constexpr int NUM_A = GATE_UP ? 2 : 1;
+    static constexpr int STAGES = GATE_UP ? 4 : 6;
+    static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 e4m3
+    static constexpr int B_BYTES = kBN8 * 128;
+    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+    static constexpr int PCOLS = NUM_A * kBN8;          // TMEM columns of one partial buffer
+    static constexpr int TMEM_COLS = GATE_UP ? 256 : 128;
+    static size_t smem_bytes(int E, int KB) {
+        return 1024 + RING_BYTES + 1024 + sizeof(float) * kBN8 * (KB + 1) + sizeof(float) * 5 * kBN8 +
+               2 * sizeof(int) * (E + 1) + 64;
+    }
+};
+
+struct Gemm8Args {
+    const int32_t *offsets, *tiles;
+    int E, MT, KB;
+    int a_rows_per_expert, up_offset;
+    const float *wscale;     // [E * rows][KB] weight scales
+    const float *xscale;     // [N][KB] activation scales of the routed rows
+    uint8_t *hq;             // gate_up: [N][F] e4m3
+    float *hs;               // gate_up: [N][F/128]
+    int F;
+    float *y;                // down: [T*K][H]
+    int H;
+    const int32_t *perm;
+    const float *topw;
+    int32_t *status;
+};
+
+__device__ __forceinline__ void epi_sync() {
+    asm volatile("bar.sync 2, %0;" ::"n"(32 * kEpi8) : "memory");
+}
+
+template <bool GATE_UP>
+__global__ void __launch_bounds__(kThreads8, 1)
+    grouped_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const Gemm8Args args) {
+    using C = Cfg8<GATE_UP>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ring = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::RING_BYTES);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *pfull = empty + C::STAGES;
+    uint64_t *pempty = pfull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pempty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *sx = reinterpret_cast<float *>(smem + C::RING_BYTES + 1024);   // [kBN8][KB+1]
+    float *amax_s = sx + kBN8 * (args.KB + 1);                            // [4][kBN8]
+    float *scale_s = amax_s + 4 * kBN8;                                   // [kBN8]
+    int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + kBN8);
+    int32_t *s_tiles = s_off + (args.E + 1);
+    const int KB = args.KB, sxp = KB + 1;
+
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&pfull[b], 1);
+            mbar_init(&pempty[b], 32 * kEpi8);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    for (int i = threadIdx.x; i <= args.E; i += blockDim.x) {
+        s_off[i] = args.offsets[i];
+        s_tiles[i] = args.tiles[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = s_tiles[args.E] * args.MT;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_x = policy_evict_last();
+            int stage = 0, armed[C::STAGES];
+            uint32_t phase = 0;
+            for (int s = 0; s < C::STAGES; ++s) armed[s] = -1;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, kBN8);
+                const int nbox = (t.nrows + 31) / 32;
+                const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * 32 * 128;
+                const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t *sA = ring + stage * C::STAGE_BYTES;
+                    uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    armed[stage] = (int)phase;
+                    tma_load_2d(sA, &tmA, &full[stage], kb * 128, arow, pol_w);
+                    if (GATE_UP)
+                        tma_load_2d(sA + C::A_BYTES, &tmA, &full[stage], kb * 128,
+                                    arow + args.up_offset, pol_w);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(sB + b * 32 * 128, &tmB, &full[stage], kb * 128,
+                                    t.row0 + b * 32, pol_x);
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+            }
+            volatile int never = 0;
+            for (int s = 0; s < C::STAGES; ++s)
+                if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
+                    atomicOr(args.status, DEV_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            int stage = 0, pb = 0;
+            uint32_t phase = 0, pphase = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, kBN8);
+                const uint32_t idesc = idesc_e4m3(kBM, (t.nrows + 15) & ~15);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag) ||
+                        !mbar_wait(&pempty[pb], pphase ^ 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(ring + stage * C::STAGE_BYTES);
+                    const uint64_t da = sdesc_sw128(sa);
+                    const uint64_t da2 = sdesc_sw128(sa + C::A_BYTES);
+                    const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES);
+                    const uint32_t d = tmem_base + pb * C::PCOLS;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        mma_e4m3_ss(d, da + 2 * k, db + 2 * k, idesc, k > 0);
+                        if (GATE_UP) mma_e4m3_ss(d + kBN8, da2 + 2 * k, db + 2 * k, idesc, k > 0);
+                    }
+                    mma_commit(&empty[stage]);
+                    mma_commit(&pfull[pb]);
+                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                    if (++pb == 2) { pb = 0; pphase ^= 1; }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+            }
+        }
+    } else {
+        const int ew = warp - 2, et = threadIdx.x - 64;
+        const int eg = warp & 3;                 // TMEM lanes [32*eg, 32*eg+32)
+        const int half = ew >> 2;                // columns [32*half, 32*half+32)
+        const int row = eg * 32 + lane;
+        int pb = 0;
+        uint32_t pphase = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, kBN8);
+            // activation scales of this tile's routed rows
+            epi_sync();
+            for (int i = et; i < t.nrows * KB; i += 32 * kEpi8) {
+                const int c = i / KB, kb = i - c * KB;
+                sx[c * sxp + kb] = __ldg(args.xscale + (size_t)(t.row0 + c) * KB + kb);
+            }
+            epi_sync();
+            const size_t wr = (size_t)t.e * args.a_rows_per_expert + t.m * kBM + row;
+            const float *wsg = args.wscale + wr * KB;
+            const float *wsu = args.wscale + (wr + args.up_offset) * KB;
+            float ag[32], au[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ag[j] = au[j] = 0.f;
+            float sg_next = __ldg(wsg), su_next = GATE_UP ? __ldg(wsu) : 0.f;
+            for (int kb = 0; kb < KB; ++kb) {
+                const float sg = sg_next, su = su_next;
+                if (kb + 1 < KB) {
+                    sg_next = __ldg(wsg + kb + 1);
+                    if (GATE_UP) su_next = __ldg(wsu + kb + 1);
+                }
+                if (ok && !mbar_wait(&pfull[pb], pphase, abort_flag)) {
+                    ok = false;
+                    *abort_flag = 1;
+                    atomicOr(args.status, DEV_TIMEOUT);
+                }
+                tc_fence_after();
+                const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + pb * C::PCOLS + half * 32;
+                uint32_t pg[32], pu[32];
+                tmem_ld32(tb, pg);
+                if (GATE_UP) tmem_ld32(tb + kBN8, pu);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&pempty[pb]);
+                if (++pb == 2) { pb = 0; pphase ^= 1; }
+                const float *sxk = sx + half * 32 * sxp + kb;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float s = sxk[j * sxp];
+                    ag[j] = fmaf(sg * s, __uint_as_float(pg[j]), ag[j]);
+                    if (GATE_UP) au[j] = fmaf(su * s, __uint_as_float(pu[j]), au[j]);
+                }
+            }
+            if (GATE_UP) {
+                // h = bf16(SiLU(g) * u) for this row (feature) and 32 routed rows
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    ag[j] = __bfloat162float(__float2bfloat16_rn(silu_f(ag[j]) * au[j]));
+                // column max of |h| over this warp's 32 rows: lane l ends with column l
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = fabsf(ag[j]);
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+                    for (int i = 0; i < o; ++i) {
+                        const bool upper = (lane & o) != 0;
+                        const float send = upper ? v[i] : v[i + o];
+                        const float keep = upper ? v[i + o] : v[i];
+                        v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
+                    }
+                }
+                amax_s[eg * kBN8 + half * 32 + lane] = v[0];
+                epi_sync();
+                if (et < kBN8) {
+                    const float m = fmaxf(fmaxf(amax_s[et], amax_s[kBN8 + et]),
+                                          fmaxf(amax_s[2 * kBN8 + et], amax_s[3 * kBN8 + et]));
+                    const int k = fp8_block_exp(m);
+                    scale_s[et] = pow2f(k);
+                    if (et < t.nrows) args.hs[(size_t)(t.row0 + et) * (args.F / 128) + t.m] = pow2f(k);
+                }
+                epi_sync();
+                uint8_t *hp = args.hq + (size_t)(t.row0 + half * 32) * args.F + t.m * kBM + row;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    if (half * 32 + j < t.nrows) {
+                        const float inv = 1.0f / scale_s[half * 32 + j];
+                        hp[(size_t)j * args.F] = (uint8_t)(e4m3x2(ag[j] * inv, 0.f) & 0xFF);
+                    }
+                }
+            } else {
+                const int c = half * 32 + lane;
+                const int my_slot = (c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
+                const float my_w = (c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
+                float *yp = args.y + t.m * kBM + row;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                    const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                    if (half * 32 + j < t.nrows) yp[(size_t)slot * args.H] = wj * ag[j];
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+template <bool GATE_UP>
+cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &b, const Gemm8Args &args,
+                        cudaStream_t st) {
+    using C = Cfg8<GATE_UP>;
+    static int attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8<GATE_UP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)C::smem_bytes(1024, kMaxKB8));
+        if (e != cudaSuccess) return e;
+        attr_done[dev & 63] = 1;
+    }
+    return launch_k(grouped_gemm_fp8<GATE_UP>, dim3(num_sms()), dim3(kThreads8),
+                    C::smem_bytes(args.E, args.KB), st, true, a, b, args);
+}
+
+}  // namespace
+
+cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
+                             const float *topw, int64_t T, int H, int F, int E, int K, uint8_t *ws,
+                             const Workspace &L, cudaStream_t st) {
+    if (H / 128 > kMaxKB8 || F / 128 > kMaxKB8) return cudaErrorInvalidValue;
+    const uint64_t N = (uint64_t)T * K;
+    CUtensorMap ta, tb, tc, td;
+    const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    if (!make_tmap(&ta, U8, 1, w13, (uint64_t)E * 2 * F, H, kBM) ||
+        !make_tmap(&tb, U8, 1, ws + L.xperm, N, H, 32) ||
+        !make_tmap(&tc, U8, 1, w2, (uint64_t)E * H, F, kBM) ||
+        !make_tmap(&td, U8, 1, ws + L.h, N, F, 32))
+        return cudaErrorInvalidValue;
+    Gemm8Args g = {};
+    g.offsets = (const int32_t *)(ws + L.offsets);
+    g.E = E;
+    g.perm = (const int32_t *)(ws + L.perm);
+    g.topw = topw;
+    g.status = (int32_t *)(ws + L.status);
+    g.hq = ws + L.h;
+    g.hs = (float *)(ws + L.hscale);
+    g.y = (float *)(ws + L.y);
+    g.F = F;
+    g.H = H;
+
+    Gemm8Args a1 = g;
+    a1.tiles = (const int32_t *)(ws + L.tiles_g);
+    a1.MT = F / kBM;
+    a1.KB = H / 128;
+    a1.a_rows_per_expert = 2 * F;
+    a1.up_offset = F;
+    a1.wscale = w13s;
+    a1.xscale = (const float *)(ws + L.xscale);
+    cudaError_t err = launch_one8<true>(ta, tb, a1, st);
+    if (err != cudaSuccess) return err;
+
+    Gemm8Args a2 = g;
+    a2.tiles = (const int32_t *)(ws + L.tiles_d);
+    a2.MT = H / kBM;
+    a2.KB = F / 128;
+    a2.a_rows_per_expert = H;
+    a2.up_offset = 0;
+    a2.wscale = w2s;
+    a2.xscale = (const float *)(ws + L.hscale);
+    return launch_one8<false>(tc, td, a2, st);
+}
+
+}  // namespace moe

@@ -15,6 +15,7 @@ namespace moe {
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBNGateUp = 128;    // routed rows (tokens) per gate_up tile
 constexpr int kBNDown = 256;      // routed rows per down tile
+constexpr int kBNFp8 = 64;        // routed rows per tile of both E4M3 GEMMs
 constexpr int kChunk = 2048;      // routing slots per histogram block
 
 // ---- workspace layout ------------------------------------------------------
@@ -64,8 +65,8 @@ bool decode_path_fits(int T, int K, int H, int F);
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 int num_sms();
 
-cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, uint8_t *ws,
-                           const Workspace &L, cudaStream_t st);
+cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, int bn_g, int bn_d,
+                           uint8_t *ws, const Workspace &L, cudaStream_t st);
 cudaError_t launch_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H, int E,
                           moe_wtype_t wt, uint8_t *ws, const Workspace &L, cudaStream_t st);
 cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, const uint8_t *ws,
@@ -74,6 +75,9 @@ cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, con
 cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float *topw, int64_t T,
                               int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
                               cudaStream_t st);
+cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
+                             const float *topw, int64_t T, int H, int F, int E, int K, uint8_t *ws,
+                             const Workspace &L, cudaStream_t st);
 cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, const uint8_t *ws,
                            const Workspace &L, void *out, cudaStream_t st);
 cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *down,

@@ -112,7 +112,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t *__restrict__ chunk_
                                                     int E, int32_t *__restrict__ counts,
                                                     int32_t *__restrict__ offsets,
                                                     int32_t *__restrict__ tiles_g,
-                                                    int32_t *__restrict__ tiles_d) {
+                                                    int32_t *__restrict__ tiles_d, int bn_g,
+                                                    int bn_d) {
     int total = 0;
     pdl_wait();
     const int e = threadIdx.x;
@@ -129,11 +130,11 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t *__restrict__ chunk_
     const int off = block_exclusive_scan(n, total);
     if (e < E) offsets[e] = off;
     if (e == 0) offsets[E] = total;
-    const int tg = (n + kBNGateUp - 1) / kBNGateUp;
+    const int tg = (n + bn_g - 1) / bn_g;
     const int tgo = block_exclusive_scan(tg, total);
     if (e < E) tiles_g[e] = tgo;
     if (e == 0) tiles_g[E] = total;
-    const int td = (n + kBNDown - 1) / kBNDown;
+    const int td = (n + bn_d - 1) / bn_d;
     const int tdo = block_exclusive_scan(td, total);
     if (e < E) tiles_d[e] = tdo;
     if (e == 0) tiles_d[E] = total;
@@ -151,7 +152,8 @@ constexpr int kSmallSlots = 1024 * kSmallRounds;
 __global__ void __launch_bounds__(1024) permute_small_kernel(
     const int32_t *__restrict__ idx, int n_slots, int E, int32_t *__restrict__ counts,
     int32_t *__restrict__ offsets, int32_t *__restrict__ tiles_g, int32_t *__restrict__ tiles_d,
-    int32_t *__restrict__ perm, int32_t *__restrict__ inv, int32_t *__restrict__ status) {
+    int32_t *__restrict__ perm, int32_t *__restrict__ inv, int32_t *__restrict__ status, int bn_g,
+    int bn_d) {
     extern __shared__ int32_t sm[];
     int32_t *wcnt = sm;                 // [32][E]
     int32_t *s_off = sm + 32 * E;       // [E+1]
@@ -200,10 +202,10 @@ __global__ void __launch_bounds__(1024) permute_small_kernel(
     const int off = block_exclusive_scan(n, total);
     if (e < E) { offsets[e] = off; s_off[e] = off; }
     if (e == 0) { offsets[E] = total; s_off[E] = total; }
-    const int tgo = block_exclusive_scan((n + kBNGateUp - 1) / kBNGateUp, total);
+    const int tgo = block_exclusive_scan((n + bn_g - 1) / bn_g, total);
     if (e < E) tiles_g[e] = tgo;
     if (e == 0) tiles_g[E] = total;
-    const int tdo = block_exclusive_scan((n + kBNDown - 1) / kBNDown, total);
+    const int tdo = block_exclusive_scan((n + bn_d - 1) / bn_d, total);
     if (e < E) tiles_d[e] = tdo;
     if (e == 0) tiles_d[E] = total;
     __syncthreads();
@@ -320,8 +322,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
 
 }  // namespace
 
-cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, uint8_t *ws,
-                           const Workspace &L, cudaStream_t st) {
+cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, int bn_g, int bn_d,
+                           uint8_t *ws, const Workspace &L, cudaStream_t st) {
     if (n_slots <= kSmallSlots) {
         const size_t smem = sizeof(int32_t) * (33 * (size_t)E + 1);
         static int attr_done[64] = {};
@@ -338,7 +340,7 @@ cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, uint8_t *
                         (int)n_slots, E, (int32_t *)(ws + L.counts), (int32_t *)(ws + L.offsets),
                         (int32_t *)(ws + L.tiles_g), (int32_t *)(ws + L.tiles_d),
                         (int32_t *)(ws + L.perm), (int32_t *)(ws + L.inv),
-                        (int32_t *)(ws + L.status));
+                        (int32_t *)(ws + L.status), bn_g, bn_d);
     }
     const int n_chunks = (int)((n_slots + kChunk - 1) / kChunk);
     int32_t *status = (int32_t *)(ws + L.status);
@@ -350,7 +352,7 @@ cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, uint8_t *
     if (err != cudaSuccess) return err;
     err = launch_k(scan_kernel, dim3(1), dim3(1024), 0, st, true, chunk_hist, n_chunks, E,
                    (int32_t *)(ws + L.counts), (int32_t *)(ws + L.offsets),
-                   (int32_t *)(ws + L.tiles_g), (int32_t *)(ws + L.tiles_d));
+                   (int32_t *)(ws + L.tiles_g), (int32_t *)(ws + L.tiles_d), bn_g, bn_d);
     if (err != cudaSuccess) return err;
     return launch_k(scatter_kernel, dim3((unsigned)((n_slots + 255) / 256)), dim3(256), 0, st, true,
                     idx, n_slots, E, (const int32_t *)chunk_hist, (const int32_t *)slot_rank,

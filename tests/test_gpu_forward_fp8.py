@@ -1,0 +1,90 @@
+"""GPU parity of the E4M3 routed-experts forward (per-(row,128) fp32 weight
+scales, activations quantised per 128 with power-of-two scales) against the
+oracle: full outputs on reduced shapes spanning several k-blocks, tiles and
+ragged tails, Zipf-skewed routing with empty experts, and sampled tokens of
+the DeepSeek-V3-like layer (H=7168, F=2048, E=256, K=8)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _helpers import assert_matches_oracle
+from mixture_experts_routed_expert_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe(cuda_dev):
+    import mixture_experts_routed_expert_b200 as m
+    return m
+
+
+def _route(lay, K, groups=8, topk_group=4, scale=2.5):
+    idx, w = oracle.route_sigmoid_grouped(inputs.np32(lay.logits), inputs.np32(lay.bias), groups,
+                                          topk_group, K, scale)
+    return torch.from_numpy(idx), torch.from_numpy(w)
+
+
+def _oracle(lay, idx, w, tokens=None):
+    """Oracle output for `tokens`; only the experts they touch go to the host
+    (their ids are remapped to 0..n-1)."""
+    E = lay.dims["E"]
+    x = lay.x if tokens is None else lay.x[tokens]
+    if tokens is not None:
+        idx, w = idx[tokens], w[tokens]
+    valid = (idx >= 0) & (idx < E)
+    used = torch.unique(idx[valid])
+    remap = torch.full((E,), -1, dtype=torch.int32)
+    remap[used.long()] = torch.arange(len(used), dtype=torch.int32)
+    ridx = torch.where(valid, remap[idx.clamp(0, E - 1).long()], torch.full_like(idx, -1))
+    sel = used.long().to(lay.w13.device)
+    return oracle.moe_forward_fp8(
+        inputs.bf16_bits(x), inputs.u8(lay.w13[sel]), inputs.np32(lay.w13_scale[sel]),
+        inputs.u8(lay.w2[sel]), inputs.np32(lay.w2_scale[sel]),
+        inputs.np32(ridx.to(torch.int32)), inputs.np32(w))
+
+
+def _run(moe, lay, idx, w, dev, fn="moe_experts_prefill"):
+    return getattr(moe, fn)(lay.x.to(dev), lay.w13.to(dev), lay.w2.to(dev), idx.to(dev), w.to(dev),
+                            idx.shape[1], gate_up_scale=lay.w13_scale.to(dev),
+                            down_scale=lay.w2_scale.to(dev))
+
+
+@pytest.mark.parametrize("T,H,F,E,K,skew", [
+    (40, 256, 256, 8, 2, None),        # two k-blocks, several tiles
+    (300, 1024, 512, 64, 8, None),     # ragged row tiles, 8 k-blocks
+    (512, 384, 384, 64, 8, 1.1),       # Zipf skew: empty experts, a hot expert (> 64 rows)
+    (3, 512, 256, 16, 4, None),        # tiny T
+])
+def test_fp8_reduced_shapes(moe, cuda_dev, T, H, F, E, K, skew):
+    lay = inputs.fp8_layer(T, seed=T + E, device="cpu", H=H, F=F, E=E, zipf=skew)
+    idx, w = _route(lay, K)
+    out = _run(moe, lay, idx, w, cuda_dev)
+    assert_matches_oracle(out, _oracle(lay, idx, w), "fp8 T=%d H=%d F=%d E=%d" % (T, H, F, E))
+
+
+def test_fp8_decode_entry(moe, cuda_dev):
+    lay = inputs.fp8_layer(2, seed=5, device="cpu", H=512, F=256, E=32)
+    idx, w = _route(lay, 8)
+    idx[1, 3] = -1
+    out = _run(moe, lay, idx, w, cuda_dev, "moe_experts_decode")
+    assert_matches_oracle(out, _oracle(lay, idx, w), "fp8 decode T=2")
+
+
+@pytest.fixture(scope="module")
+def dsv3_weights(cuda_dev):
+    return inputs.fp8_weights(seed=0, device=cuda_dev)
+
+
+@pytest.mark.parametrize("T", [128, 1])
+def test_fp8_dsv3_sampled(moe, cuda_dev, dsv3_weights, T):
+    lay = inputs.fp8_layer(T, seed=T, device="cpu", weights=dsv3_weights)
+    idx, w = _route(lay, 8)
+    out = _run(moe, lay, idx, w, cuda_dev)
+    tokens = torch.arange(T) if T <= 4 else torch.from_numpy(
+        np.random.default_rng(T).choice(T, 4, replace=False))
+    assert_matches_oracle(out[tokens.to(out.device)], _oracle(lay, idx, w, tokens),
+                          "fp8 DSV3 T=%d sampled" % T)
+    out2 = _run(moe, lay, idx, w, cuda_dev)
+    assert torch.equal(out, out2), "fp8 path is not deterministic"
