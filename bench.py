@@ -262,6 +262,38 @@ def run_ours(args):
         tc_frac=round(t_tc / us, 3), hbm_frac=round(t_hbm / us, 3),
         roofline_frac=round(max(t_hbm, t_tc) / us, 3), bound="hbm" if t_hbm > t_tc else "tensor")
     del g
+    # ---- DeepSeek-V3-like FP8 layer: group-sigmoid router + E4M3 experts ----
+    fp8_w = inputs.fp8_weights(seed=0, device=dev)
+    D = inputs.DSV3_FP8
+    for T in (128, 1):
+        lay = inputs.fp8_layer(T, seed=T, device=dev, weights=fp8_w)
+        idx = torch.empty(T, D["K"], dtype=torch.int32, device=dev)
+        tw = torch.empty(T, D["K"], dtype=torch.float32, device=dev)
+        out = torch.empty(T, D["H"], dtype=torch.bfloat16, device=dev)
+        wsz = moe.moe_experts_workspace_size(T, D["H"], D["F"], D["E"], D["K"], 1, False)
+        ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+
+        def call(lay=lay, idx=idx, tw=tw, out=out, ws=ws):
+            moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"], D["topk_group"],
+                                          D["K"], D["scale"], top_k_index=idx, top_k_weights=tw)
+            moe.moe_experts_prefill(lay.x, lay.w13, lay.w2, idx, tw, D["K"],
+                                    gate_up_scale=lay.w13_scale, down_scale=lay.w2_scale,
+                                    out=out, workspace=ws)
+        t, g = time_graph(call, args.steps, args.warmup)
+        us = float(np.mean(t))
+        n_t = len(set(idx.cpu().reshape(-1).tolist()))
+        per_expert = (2 * D["F"] * D["H"] + D["H"] * D["F"]) + 4 * (2 * D["F"] * D["H"] // 128 + D["H"] * D["F"] // 128)
+        byts = n_t * per_expert + T * D["H"] * 4 + T * D["E"] * 4
+        flops = 6 * T * D["K"] * D["H"] * D["F"]
+        t_hbm = byts / (peaks["hbm"] * 1e3)
+        t_tc = flops / (2 * peaks["bf16"] * 1e6)
+        breakdown["fp8_dsv3_T%d" % T] = dict(
+            us=round(us, 2), touched_experts=n_t, gbs=round(byts / us / 1e3, 1),
+            tflops=round(flops / us / 1e6, 1), hbm_frac=round(t_hbm / us, 3),
+            tc_frac=round(t_tc / us, 3), roofline_frac=round(max(t_hbm, t_tc) / us, 3),
+            bound="hbm" if t_hbm > t_tc else "tensor", includes="router + quantise + experts")
+        del g
+    del fp8_w
 
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "decode_ocr2_T1_traffic.json")
@@ -310,6 +342,25 @@ def run_only(args):
     from mixture_experts_routed_expert_b200 import inputs
 
     dev = torch.device("cuda", 0)
+    if args.only in ("fp8_128", "fp8_small"):
+        # fp8_small: the DeepSeek-V3 expert shapes with 32 experts (1.5 GB of
+        # weights) and 16 tokens, small enough for multi-pass profiler captures
+        D = dict(inputs.DSV3_FP8)
+        T = 128
+        if args.only == "fp8_small":
+            D["E"], T = 32, 16
+        wts = inputs.fp8_weights(seed=0, device=dev, E=D["E"])
+        lay = inputs.fp8_layer(T, seed=T, device=dev, E=D["E"], weights=wts)
+        flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        for i in range(args.warmup + args.steps):
+            flush_w.fill_(i & 0xFF)
+            idx, tw = moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"],
+                                                    D["topk_group"], D["K"], D["scale"])
+            out = moe.moe_experts_prefill(lay.x, lay.w13, lay.w2, idx, tw, D["K"],
+                                          gate_up_scale=lay.w13_scale, down_scale=lay.w2_scale)
+        torch.cuda.synchronize()
+        print("ok", args.only, float(out.float().abs().sum()))
+        return
     T = {"decode1": 1, "decode4": 4, "prefill2048": 2048}[args.only]
     fn = moe.moe_experts_prefill if args.only.startswith("prefill") else moe.moe_experts_decode
     lay = inputs.ocr2_layer(T, seed=T, device=dev)
@@ -393,7 +444,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048"], default=None,
+    ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048", "fp8_128", "fp8_small"],
+                    default=None,
                     help="run just W+K eager calls of one workload (for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
