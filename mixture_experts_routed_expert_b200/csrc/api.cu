@@ -52,13 +52,10 @@ bool dims_ok(int64_t T, int H, int F, int E, int K) {
 
 Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t wt) {
     const int64_t N = T * K;
-    const int64_t C = (N + kChunk - 1) / kChunk;
     const size_t eb = (wt == MOE_W_BF16) ? 2 : 1;
     Workspace L;
     Bump b;
     L.status = b.take(16);
-    L.chunk_hist = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(C, 1) * E);
-    L.slot_rank = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(C * kChunk, 1));
     L.counts = b.take(sizeof(int32_t) * E);
     L.offsets = b.take(sizeof(int32_t) * (E + 1));
     L.tiles_g = b.take(sizeof(int32_t) * (E + 1));
@@ -123,9 +120,8 @@ moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const in
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     const int64_t N = (int64_t)T * K;
     const bool fp8 = (wt == MOE_W_FP8_E4M3);
-    cudaError_t e = fp8 ? launch_permute(idx, N, E, kBNFp8, kBNFp8, wsb, L, st)
-                        : launch_permute(idx, N, E, kBNGateUp, kBNDown, wsb, L, st);
-    if (e == cudaSuccess) e = launch_gather(x, idx, N, K, H, E, wt, wsb, L, st);
+    cudaError_t e = fp8 ? launch_permute_gather(x, idx, N, K, H, E, kBNFp8, kBNFp8, wt, wsb, L, st)
+                        : launch_permute_gather(x, idx, N, K, H, E, kBNGateUp, kBNDown, wt, wsb, L, st);
     if (e == cudaSuccess)
         e = fp8 ? launch_gemms_fp8(gu, gus, dn, dns, w, T, H, F, E, K, wsb, L, st)
                 : launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st);

@@ -16,13 +16,10 @@ constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBNGateUp = 128;    // routed rows (tokens) per gate_up tile
 constexpr int kBNDown = 256;      // routed rows per down tile
 constexpr int kBNFp8 = 64;        // routed rows per tile of both E4M3 GEMMs
-constexpr int kChunk = 2048;      // routing slots per histogram block
 
 // ---- workspace layout ------------------------------------------------------
 struct Workspace {
     size_t status;        // int32 device status word
-    size_t chunk_hist;    // [C][E] int32: per-chunk counts, then per-chunk bases
-    size_t slot_rank;     // [N] int32 rank of a slot among its chunk's slots of one expert
     size_t counts;        // [E] int32
     size_t offsets;       // [E+1] int32
     size_t tiles_g;       // [E+1] int32 prefix of gate_up row tiles per expert
@@ -67,8 +64,9 @@ int num_sms();
 
 cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, int bn_g, int bn_d,
                            uint8_t *ws, const Workspace &L, cudaStream_t st);
-cudaError_t launch_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H, int E,
-                          moe_wtype_t wt, uint8_t *ws, const Workspace &L, cudaStream_t st);
+cudaError_t launch_permute_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H,
+                                  int E, int bn_g, int bn_d, moe_wtype_t wt, uint8_t *ws,
+                                  const Workspace &L, cudaStream_t st);
 cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, const uint8_t *ws,
                                  const Workspace &L, int32_t *counts, int32_t *offsets,
                                  int32_t *perm, int32_t *inv, cudaStream_t st);

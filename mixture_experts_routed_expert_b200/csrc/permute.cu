@@ -1,6 +1,7 @@
-// permute.cu -- S3 (expert histogram, prefix scan, stable permutation of the
-// routing slots, gather of the routed activation rows) and S6 (fixed-order
-// top-K combine) for the prefill path.
+// permute.cu -- S3 (expert histogram, offsets, stable permutation of the
+// routing slots and gather of the routed activation rows, E4M3-quantised on
+// the way for the FP8 path) and S6 (fixed-order top-K combine) of the prefill
+// path.
 //
 // The model card ("deepseek-ocr2-moe-experts", description) computes the
 // routed experts as a grouped GEMM followed by a router-weight scale and a
@@ -9,6 +10,11 @@
 //
 // Slot s = t*K + k.  Slots of one expert are placed in ascending slot order,
 // so every integer output is unique and bit-exact.
+//
+// One kernel does S3 without any inter-block communication: every block
+// recounts the whole routing (T*K int32, read from L2) to get the expert
+// offsets and the number of earlier slots of each expert before its own chunk,
+// ranks its chunk's slots stably, writes perm / inv and gathers its rows.
 #include "common.cuh"
 #include "internal.h"
 
@@ -16,284 +22,173 @@ namespace moe {
 
 namespace {
 
-constexpr int kHistWarps = 8;                       // 256 threads per histogram block
-constexpr int kSlotsPerWarp = kChunk / kHistWarps;  // 256 consecutive slots per warp
+constexpr int kPThreads = 256;
+constexpr int kPWarps = kPThreads / 32;
 
-// Block c handles slots [c*kChunk, (c+1)*kChunk).  Each warp walks its 256
-// slots in order, 32 at a time; lanes routed to the same expert find each
-// other with match.any and take consecutive ranks.  Output: per-block expert
-// counts and, per slot, its rank among the block's earlier slots of the same
-// expert.  smem: kHistWarps x E counters.
-__global__ void __launch_bounds__(256) hist_kernel(const int32_t *__restrict__ idx, int64_t n_slots,
-                                                   int E, int32_t *__restrict__ chunk_hist,
-                                                   int32_t *__restrict__ slot_rank,
-                                                   int32_t *__restrict__ status) {
-    extern __shared__ int32_t wcnt[];  // [kHistWarps][E]
-    const int warp = threadIdx.x >> 5, lane = lane_id();
-    if (blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
-    for (int i = threadIdx.x; i < kHistWarps * E; i += blockDim.x) wcnt[i] = 0;
-    __syncthreads();
-    const int64_t base = (int64_t)blockIdx.x * kChunk + (int64_t)warp * kSlotsPerWarp;
-    int local[kSlotsPerWarp / 32];
-    int ex[kSlotsPerWarp / 32];
-    const unsigned lt_mask = (1u << lane) - 1u;
-#pragma unroll
-    for (int r = 0; r < kSlotsPerWarp / 32; ++r) {
-        const int64_t s = base + r * 32 + lane;
-        int e = (s < n_slots) ? __ldg(idx + s) : -1;
-        const bool valid = (e >= 0 && e < E);
-        if (!valid) e = -1;
-        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-        const int rank = __popc(peers & lt_mask);
-        const int prior = valid ? wcnt[warp * E + e] : 0;
-        __syncwarp();
-        if (valid && rank == 0) wcnt[warp * E + e] = prior + __popc(peers);
-        __syncwarp();
-        local[r] = prior + rank;
-        ex[r] = e;
-    }
-    __syncthreads();
-    // exclusive scan over the warps of each expert; block totals to global
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
-#pragma unroll
-        for (int w = 0; w < kHistWarps; ++w) {
-            const int v = wcnt[w * E + e];
-            wcnt[w * E + e] = run;
-            run += v;
-        }
-        chunk_hist[(int64_t)blockIdx.x * E + e] = run;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int r = 0; r < kSlotsPerWarp / 32; ++r) {
-        const int64_t s = base + r * 32 + lane;
-        if (ex[r] >= 0) slot_rank[s] = wcnt[warp * E + ex[r]] + local[r];
-    }
-    pdl_launch_dependents();
-}
-
-// Block-wide exclusive scan of one int per thread (blockDim.x == 1024);
-// `total` receives the sum over the block.
-__device__ int block_exclusive_scan(int v, int &total) {
-    __shared__ int warp_sums[32];
-    __shared__ int block_total;
-    const int lane = lane_id(), warp = threadIdx.x >> 5;
-    int incl = v;
+// Exclusive scan of n ints in place (n <= 4096) by one block of kPThreads
+// threads; returns the total.  Each thread scans a contiguous run.
+__device__ int block_scan_inplace(int32_t *v, int n) {
+    __shared__ int warp_tot[kPWarps];
+    __shared__ int grand;
+    const int t = threadIdx.x, lane = lane_id(), warp = t >> 5;
+    const int per = (n + kPThreads - 1) / kPThreads;
+    const int b = min(n, t * per), e = min(n, b + per);
+    int local = 0;
+    for (int i = b; i < e; ++i) local += v[i];
+    int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += n;
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
     }
-    if (lane == 31) warp_sums[warp] = incl;
+    if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        const int ws = warp_sums[lane];
-        int wincl = ws;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xFFFFFFFFu, wincl, o);
-            if (lane >= o) wincl += n;
+    if (t == 0) {
+        int run = 0;
+        for (int w = 0; w < kPWarps; ++w) {
+            const int x = warp_tot[w];
+            warp_tot[w] = run;
+            run += x;
         }
-        warp_sums[lane] = wincl - ws;
-        if (lane == 31) block_total = wincl;
+        grand = run;
     }
     __syncthreads();
-    const int r = warp_sums[warp] + incl - v;
-    total = block_total;
+    int run = warp_tot[warp] + incl - local;
+    for (int i = b; i < e; ++i) {
+        const int x = v[i];
+        v[i] = run;
+        run += x;
+    }
+    const int total = grand;
     __syncthreads();
-    return r;
+    return total;
 }
 
-// One block of 1024 threads, one expert per thread (E <= 1024):
-// per-chunk counts -> per-chunk exclusive bases (in place), expert counts,
-// expert offsets, and prefix sums of row tiles for both grouped GEMMs.
-__global__ void __launch_bounds__(1024) scan_kernel(int32_t *__restrict__ chunk_hist, int n_chunks,
-                                                    int E, int32_t *__restrict__ counts,
-                                                    int32_t *__restrict__ offsets,
-                                                    int32_t *__restrict__ tiles_g,
-                                                    int32_t *__restrict__ tiles_d, int bn_g,
-                                                    int bn_d) {
-    int total = 0;
-    pdl_wait();
-    const int e = threadIdx.x;
-    int run = 0;
-    if (e < E) {
-        for (int c = 0; c < n_chunks; ++c) {
-            const int v = chunk_hist[(int64_t)c * E + e];
-            chunk_hist[(int64_t)c * E + e] = run;
-            run += v;
-        }
-        counts[e] = run;
-    }
-    const int n = (e < E) ? run : 0;
-    const int off = block_exclusive_scan(n, total);
-    if (e < E) offsets[e] = off;
-    if (e == 0) offsets[E] = total;
-    const int tg = (n + bn_g - 1) / bn_g;
-    const int tgo = block_exclusive_scan(tg, total);
-    if (e < E) tiles_g[e] = tgo;
-    if (e == 0) tiles_g[E] = total;
-    const int td = (n + bn_d - 1) / bn_d;
-    const int tdo = block_exclusive_scan(td, total);
-    if (e < E) tiles_d[e] = tdo;
-    if (e == 0) tiles_d[E] = total;
-    pdl_launch_dependents();
-}
-
-// Whole permutation in one block of 1024 threads, for up to
-// kSmallSlots slots: warp w takes slots [w*R, (w+1)*R), R = 32*rounds, and
-// ranks them as hist_kernel does; then per-expert bases over the warps,
-// expert counts / offsets / tile prefixes, and the final positions.
-// smem: 32 x E counters + E+1 offsets.
-constexpr int kSmallRounds = 16;
-constexpr int kSmallSlots = 1024 * kSmallRounds;
-
-__global__ void __launch_bounds__(1024) permute_small_kernel(
-    const int32_t *__restrict__ idx, int n_slots, int E, int32_t *__restrict__ counts,
-    int32_t *__restrict__ offsets, int32_t *__restrict__ tiles_g, int32_t *__restrict__ tiles_d,
-    int32_t *__restrict__ perm, int32_t *__restrict__ inv, int32_t *__restrict__ status, int bn_g,
-    int bn_d) {
-    extern __shared__ int32_t sm[];
-    int32_t *wcnt = sm;                 // [32][E]
-    int32_t *s_off = sm + 32 * E;       // [E+1]
-    const int warp = threadIdx.x >> 5, lane = lane_id();
-    if (threadIdx.x == 0) *status = 0;
-    for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
-    const int rounds = (n_slots + 1023) / 1024;
-    const int base = warp * rounds * 32;
-    int loc[kSmallRounds], ex[kSmallRounds];
-#pragma unroll
-    for (int r = 0; r < kSmallRounds; ++r) {
-        ex[r] = -1;
-        const int s = base + r * 32 + lane;
-        if (r < rounds && s < n_slots) {
-            const int e = __ldg(idx + s);
-            if (e >= 0 && e < E) ex[r] = e;
-        }
-    }
+// MODE 0: permutation only; 1: + bf16 row gather; 2: + gather with block-128
+// E4M3 quantisation (the rule of quantize_fp8_block128).
+// Block b handles slots [b*chunk, (b+1)*chunk), chunk <= kPThreads.
+// Dynamic shared memory: cnt_all[E+1], cnt_before[E], wc[kPWarps][E], tiles[E+1].
+template <int MODE>
+__global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
+    const int32_t *__restrict__ idx, int n_slots, int E, int K, int H, int chunk, int bn_g,
+    int bn_d, const uint4 *__restrict__ x, void *__restrict__ xperm, float *__restrict__ xscale,
+    int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ tiles_g,
+    int32_t *__restrict__ tiles_d, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
+    int32_t *__restrict__ status) {
+    extern __shared__ int32_t psm[];
+    int32_t *cnt_all = psm;                 // [E+1] -> exclusive offsets
+    int32_t *cnt_bef = cnt_all + (E + 1);   // [E] slots of e before this chunk
+    int32_t *wc = cnt_bef + E;              // [kPWarps][E] per-warp counts in the chunk
+    int32_t *tl = wc + kPWarps * E;         // [E+1] tile counts (block 0)
+    __shared__ int32_t pos_s[kPThreads];
+    const int t = threadIdx.x, lane = lane_id(), warp = t >> 5;
+    const int c0 = blockIdx.x * chunk;
+    for (int i = t; i < (2 + kPWarps) * E + 1; i += kPThreads) psm[i] = 0;
     __syncthreads();
-    const unsigned lt_mask = (1u << lane) - 1u;
+    // 1. global counts and counts before this chunk (integer smem atomics);
+    //    16-byte index loads, eight in flight per thread
+    const int n4 = (reinterpret_cast<uintptr_t>(idx) & 15) == 0 ? n_slots / 4 : 0;
+    const int4 *idx4 = reinterpret_cast<const int4 *>(idx);
+    for (int q0 = 0; q0 < n4; q0 += 8 * kPThreads) {
+        int4 ev[8];
 #pragma unroll
-    for (int r = 0; r < kSmallRounds; ++r) {
-        if (r < rounds) {
-            const int e = ex[r];
-            const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-            const int rank = __popc(peers & lt_mask);
-            const int prior = (e >= 0) ? wcnt[warp * E + e] : 0;
-            __syncwarp();
-            if (e >= 0 && rank == 0) wcnt[warp * E + e] = prior + __popc(peers);
-            __syncwarp();
-            loc[r] = prior + rank;
+        for (int u = 0; u < 8; ++u) {
+            const int q = q0 + u * kPThreads + t;
+            ev[u] = q < n4 ? __ldg(idx4 + q) : make_int4(-1, -1, -1, -1);
         }
-    }
-    __syncthreads();
-    int n = 0;
-    const int e = threadIdx.x;
-    if (e < E) {
-        for (int w = 0; w < 32; ++w) {
-            const int v = wcnt[w * E + e];
-            wcnt[w * E + e] = n;
-            n += v;
-        }
-        counts[e] = n;
-    }
-    int total = 0;
-    const int off = block_exclusive_scan(n, total);
-    if (e < E) { offsets[e] = off; s_off[e] = off; }
-    if (e == 0) { offsets[E] = total; s_off[E] = total; }
-    const int tgo = block_exclusive_scan((n + bn_g - 1) / bn_g, total);
-    if (e < E) tiles_g[e] = tgo;
-    if (e == 0) tiles_g[E] = total;
-    const int tdo = block_exclusive_scan((n + bn_d - 1) / bn_d, total);
-    if (e < E) tiles_d[e] = tdo;
-    if (e == 0) tiles_d[E] = total;
-    __syncthreads();
 #pragma unroll
-    for (int r = 0; r < kSmallRounds; ++r) {
-        const int s = base + r * 32 + lane;
-        if (r < rounds && s < n_slots) {
-            if (ex[r] >= 0) {
-                const int pos = s_off[ex[r]] + wcnt[warp * E + ex[r]] + loc[r];
-                perm[pos] = s;
-                inv[s] = pos;
-            } else {
-                inv[s] = -1;
+        for (int u = 0; u < 8; ++u) {
+            const int s4 = 4 * (q0 + u * kPThreads + t);
+            const int ee[4] = {ev[u].x, ev[u].y, ev[u].z, ev[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (ee[j] >= 0 && ee[j] < E) {
+                    atomicAdd(&cnt_all[ee[j]], 1);
+                    if (s4 + j < c0) atomicAdd(&cnt_bef[ee[j]], 1);
+                }
             }
         }
     }
-    for (int p = s_off[E] + threadIdx.x; p < n_slots; p += blockDim.x) perm[p] = -1;
-    pdl_launch_dependents();
-}
-
-// Final slot positions.  One thread per slot; also fills perm entries past
-// offsets[E] (slots whose expert id is out of range) with -1.
-__global__ void __launch_bounds__(256) scatter_kernel(
-    const int32_t *__restrict__ idx, int64_t n_slots, int E, const int32_t *__restrict__ chunk_hist,
-    const int32_t *__restrict__ slot_rank, const int32_t *__restrict__ offsets,
-    int32_t *__restrict__ perm, int32_t *__restrict__ inv) {
-    pdl_wait();
-    const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (s >= n_slots) return;
-    const int e = __ldg(idx + s);
-    if (e >= 0 && e < E) {
-        const int pos = offsets[e] + chunk_hist[(s / kChunk) * E + e] + slot_rank[s];
-        perm[pos] = (int32_t)s;
-        inv[s] = pos;
-    } else {
-        inv[s] = -1;
-    }
-    if (s >= offsets[E]) perm[s] = -1;
-    pdl_launch_dependents();
-}
-
-// Gather of routed activation rows into expert order: xperm[inv[s]] = x[s/K].
-// One warp per slot, 16-byte vectors.
-__global__ void __launch_bounds__(256) gather_bf16_kernel(const uint4 *__restrict__ x,
-                                                          const int32_t *__restrict__ inv,
-                                                          int64_t n_slots, int K, int H,
-                                                          uint4 *__restrict__ xperm) {
-    pdl_wait();
-    const int64_t s = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (s >= n_slots) return;
-    const int pos = inv[s];
-    if (pos < 0) return;
-    const int nv = H / 8;
-    const uint4 *src = x + (s / K) * nv;
-    uint4 *dst = xperm + (int64_t)pos * nv;
-    for (int v = lane_id(); v < nv; v += 32) dst[v] = __ldg(src + v);
-    pdl_launch_dependents();
-}
-
-// Gather + block-128 E4M3 quantisation of the routed activation rows
-// (the rule of quantize_fp8_block128).  One warp per slot; 16 lanes cover a
-// block of 128 values (8 per lane).
-__global__ void __launch_bounds__(256) gather_fp8_kernel(const uint4 *__restrict__ x,
-                                                         const int32_t *__restrict__ inv,
-                                                         int64_t n_slots, int K, int H,
-                                                         uint2 *__restrict__ xq,
-                                                         float *__restrict__ xs) {
-    pdl_wait();
-    const int64_t s = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (s >= n_slots) return;
-    const int pos = inv[s];
-    if (pos < 0) return;
-    const int lane = lane_id();
-    const int nv = H / 8;
-    const uint4 *src = x + (s / K) * nv;
-    for (int v0 = 0; v0 < nv; v0 += 32) {
-        const int v = v0 + lane;
-        const bool on = v < nv;
-        float f[8];
-        unpack_bf16x8(on ? __ldg(src + v) : make_uint4(0, 0, 0, 0), f);
-        float sc;
-        const uint2 q = quant8_e4m3(f, sc);
-        if (on) {
-            xq[(int64_t)pos * nv + v] = q;
-            if ((lane & 15) == 0) xs[(int64_t)pos * (H / 128) + v / 16] = sc;
+    for (int s = 4 * n4 + t; s < n_slots; s += kPThreads) {   // tail (n_slots % 4)
+        const int e = __ldg(idx + s);
+        if (e >= 0 && e < E) {
+            atomicAdd(&cnt_all[e], 1);
+            if (s < c0) atomicAdd(&cnt_bef[e], 1);
         }
     }
-    pdl_launch_dependents();
+    __syncthreads();
+    if (blockIdx.x == 0)
+        for (int i = t; i < E; i += kPThreads) {
+            counts[i] = cnt_all[i];
+            tl[i] = cnt_all[i];
+        }
+    const int total = block_scan_inplace(cnt_all, E);   // cnt_all -> offsets
+    // 2. stable rank of each slot of the chunk among the chunk's slots of its expert
+    const int s = c0 + t;
+    const bool mine = t < chunk && s < n_slots;
+    int e = mine ? __ldg(idx + s) : -1;
+    if (e < 0 || e >= E) e = -1;
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank_w = __popc(peers & ((1u << lane) - 1u));
+    if (e >= 0 && rank_w == 0) wc[warp * E + e] = __popc(peers);
+    __syncthreads();
+    int pos = -1;
+    if (e >= 0) {
+        int r = rank_w;
+        for (int w = 0; w < warp; ++w) r += wc[w * E + e];
+        pos = cnt_all[e] + cnt_bef[e] + r;
+        perm[pos] = s;
+    }
+    if (mine) inv[s] = pos;
+    pos_s[t] = mine ? pos : -1;
+    if (blockIdx.x == 0) {
+        if (t == 0) {
+            *status = 0;
+            offsets[E] = total;
+        }
+        for (int i = t; i < E; i += kPThreads) offsets[i] = cnt_all[i];
+        for (int p = total + t; p < n_slots; p += kPThreads) perm[p] = -1;
+        // row-tile prefixes for both GEMMs
+        __syncthreads();
+        for (int i = t; i < E; i += kPThreads) tl[i] = (tl[i] + bn_g - 1) / bn_g;
+        __syncthreads();
+        const int tg = block_scan_inplace(tl, E);
+        for (int i = t; i < E; i += kPThreads) tiles_g[i] = tl[i];
+        if (t == 0) tiles_g[E] = tg;
+        __syncthreads();
+        for (int i = t; i < E; i += kPThreads) tl[i] = (counts[i] + bn_d - 1) / bn_d;
+        __syncthreads();
+        const int td = block_scan_inplace(tl, E);
+        for (int i = t; i < E; i += kPThreads) tiles_d[i] = tl[i];
+        if (t == 0) tiles_d[E] = td;
+    }
+    __syncthreads();
+    if (MODE == 0) return;
+    // 3. gather the chunk's rows: one warp per row, 16-byte vectors
+    const int nv = H / 8;
+    for (int r = warp; r < chunk; r += kPWarps) {
+        const int p = pos_s[r];
+        if (p < 0) continue;
+        const uint4 *src = x + (size_t)((c0 + r) / K) * nv;
+        if (MODE == 1) {
+            uint4 *dst = reinterpret_cast<uint4 *>(xperm) + (size_t)p * nv;
+            for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+        } else {
+            uint2 *dst = reinterpret_cast<uint2 *>(xperm) + (size_t)p * nv;
+            for (int v0 = 0; v0 < nv; v0 += 32) {
+                const int v = v0 + lane;
+                const bool on = v < nv;
+                float f[8];
+                unpack_bf16x8(on ? __ldg(src + v) : make_uint4(0, 0, 0, 0), f);
+                float sc;
+                const uint2 q = quant8_e4m3(f, sc);   // every lane takes part
+                if (on) {
+                    dst[v] = q;
+                    if ((lane & 15) == 0) xscale[(size_t)p * (H / 128) + v / 16] = sc;
+                }
+            }
+        }
+    }
 }
 
 // S6: out[t, j] = bf16( sum_{k in order} y[t*K + k, j] ) over slots with a
@@ -320,57 +215,46 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
     out[t * nv + v] = o;
 }
 
+template <int MODE>
+cudaError_t launch_pg(const void *x, const int32_t *idx, int64_t n_slots, int K, int H, int E,
+                      int bn_g, int bn_d, uint8_t *ws, const Workspace &L, cudaStream_t st) {
+    const size_t smem = sizeof(int32_t) * ((3 + kPWarps) * (size_t)E + 2);
+    static int attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_done[dev & 63]) {
+        cudaError_t e = cudaFuncSetAttribute(permute_gather_kernel<MODE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(sizeof(int32_t) * ((3 + kPWarps) * 1024 + 2)));
+        if (e != cudaSuccess) return e;
+        attr_done[dev & 63] = 1;
+    }
+    // about two blocks per SM for the gather; at least 128 slots per block
+    // once the redundant recount of all slots becomes the larger cost
+    int chunk = kPThreads;
+    const int64_t floor_chunk = n_slots > 32768 ? 128 : 8;
+    while (chunk > floor_chunk && n_slots / chunk < 2 * num_sms()) chunk /= 2;
+    const unsigned blocks = (unsigned)((n_slots + chunk - 1) / chunk);
+    return launch_k(permute_gather_kernel<MODE>, dim3(blocks), dim3(kPThreads), smem, st, false,
+                    idx, (int)n_slots, E, K, H, chunk, bn_g, bn_d, (const uint4 *)x,
+                    (void *)(ws + L.xperm), (float *)(ws + L.xscale), (int32_t *)(ws + L.counts),
+                    (int32_t *)(ws + L.offsets), (int32_t *)(ws + L.tiles_g),
+                    (int32_t *)(ws + L.tiles_d), (int32_t *)(ws + L.perm), (int32_t *)(ws + L.inv),
+                    (int32_t *)(ws + L.status));
+}
+
 }  // namespace
 
 cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, int bn_g, int bn_d,
                            uint8_t *ws, const Workspace &L, cudaStream_t st) {
-    if (n_slots <= kSmallSlots) {
-        const size_t smem = sizeof(int32_t) * (33 * (size_t)E + 1);
-        static int attr_done[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (!attr_done[dev & 63]) {
-            cudaError_t e = cudaFuncSetAttribute(permute_small_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)(sizeof(int32_t) * (33 * 1024 + 1)));
-            if (e != cudaSuccess) return e;
-            attr_done[dev & 63] = 1;
-        }
-        return launch_k(permute_small_kernel, dim3(1), dim3(1024), smem, st, false, idx,
-                        (int)n_slots, E, (int32_t *)(ws + L.counts), (int32_t *)(ws + L.offsets),
-                        (int32_t *)(ws + L.tiles_g), (int32_t *)(ws + L.tiles_d),
-                        (int32_t *)(ws + L.perm), (int32_t *)(ws + L.inv),
-                        (int32_t *)(ws + L.status), bn_g, bn_d);
-    }
-    const int n_chunks = (int)((n_slots + kChunk - 1) / kChunk);
-    int32_t *status = (int32_t *)(ws + L.status);
-    int32_t *chunk_hist = (int32_t *)(ws + L.chunk_hist);
-    int32_t *slot_rank = (int32_t *)(ws + L.slot_rank);
-    const size_t hsmem = sizeof(int32_t) * kHistWarps * E;
-    cudaError_t err = launch_k(hist_kernel, dim3(n_chunks), dim3(256), hsmem, st, false, idx,
-                               n_slots, E, chunk_hist, slot_rank, status);
-    if (err != cudaSuccess) return err;
-    err = launch_k(scan_kernel, dim3(1), dim3(1024), 0, st, true, chunk_hist, n_chunks, E,
-                   (int32_t *)(ws + L.counts), (int32_t *)(ws + L.offsets),
-                   (int32_t *)(ws + L.tiles_g), (int32_t *)(ws + L.tiles_d), bn_g, bn_d);
-    if (err != cudaSuccess) return err;
-    return launch_k(scatter_kernel, dim3((unsigned)((n_slots + 255) / 256)), dim3(256), 0, st, true,
-                    idx, n_slots, E, (const int32_t *)chunk_hist, (const int32_t *)slot_rank,
-                    (const int32_t *)(ws + L.offsets), (int32_t *)(ws + L.perm),
-                    (int32_t *)(ws + L.inv));
+    return launch_pg<0>(nullptr, idx, n_slots, 1, 128, E, bn_g, bn_d, ws, L, st);
 }
 
-cudaError_t launch_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H, int E,
-                          moe_wtype_t wt, uint8_t *ws, const Workspace &L, cudaStream_t st) {
-    (void)idx;
-    (void)E;
-    const dim3 grid((unsigned)((n_slots + 7) / 8));
-    if (wt == MOE_W_BF16)
-        return launch_k(gather_bf16_kernel, grid, dim3(256), 0, st, true, (const uint4 *)x,
-                        (const int32_t *)(ws + L.inv), n_slots, K, H, (uint4 *)(ws + L.xperm));
-    return launch_k(gather_fp8_kernel, grid, dim3(256), 0, st, true, (const uint4 *)x,
-                    (const int32_t *)(ws + L.inv), n_slots, K, H, (uint2 *)(ws + L.xperm),
-                    (float *)(ws + L.xscale));
+cudaError_t launch_permute_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H,
+                                  int E, int bn_g, int bn_d, moe_wtype_t wt, uint8_t *ws,
+                                  const Workspace &L, cudaStream_t st) {
+    if (wt == MOE_W_BF16) return launch_pg<1>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
+    return launch_pg<2>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
 }
 
 cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, const uint8_t *ws,
