@@ -280,35 +280,64 @@ def run_ours(args):
     # ---- DeepSeek-V3-like FP8 layer: group-sigmoid router + E4M3 experts ----
     fp8_w = inputs.fp8_weights(seed=0, device=dev)
     D = inputs.DSV3_FP8
-    for T in (128, 1):
-        lay = inputs.fp8_layer(T, seed=T, device=dev, weights=fp8_w)
+    per_expert_fp8 = (3 * D["F"] * D["H"]) + 4 * (3 * D["F"] * D["H"] // 128)
+
+    def fp8_entry(T, zipf, steps):
+        lay = inputs.fp8_layer(T, seed=T, device=dev, weights=fp8_w, zipf=zipf)
         idx = torch.empty(T, D["K"], dtype=torch.int32, device=dev)
         tw = torch.empty(T, D["K"], dtype=torch.float32, device=dev)
         out = torch.empty(T, D["H"], dtype=torch.bfloat16, device=dev)
         wsz = moe.moe_experts_workspace_size(T, D["H"], D["F"], D["E"], D["K"], 1, False)
         ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
 
-        def call(lay=lay, idx=idx, tw=tw, out=out, ws=ws):
+        def call():
             moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"], D["topk_group"],
                                           D["K"], D["scale"], top_k_index=idx, top_k_weights=tw)
             moe.moe_experts_prefill(lay.x, lay.w13, lay.w2, idx, tw, D["K"],
                                     gate_up_scale=lay.w13_scale, down_scale=lay.w2_scale,
                                     out=out, workspace=ws)
-        t, g = time_graph(call, args.steps, args.warmup)
+        t, g = time_graph(call, steps, args.warmup)
         us = float(np.mean(t))
         n_t = len(set(idx.cpu().reshape(-1).tolist()))
-        per_expert = (2 * D["F"] * D["H"] + D["H"] * D["F"]) + 4 * (2 * D["F"] * D["H"] // 128 + D["H"] * D["F"] // 128)
-        byts = n_t * per_expert + T * D["H"] * 4 + T * D["E"] * 4
+        byts = n_t * per_expert_fp8 + T * D["H"] * 4 + T * D["E"] * 4
         flops = 6 * T * D["K"] * D["H"] * D["F"]
         t_hbm = byts / (peaks["hbm"] * 1e3)
         t_tc = flops / (2 * peaks["bf16"] * 1e6)
-        breakdown["fp8_dsv3_T%d" % T] = dict(
-            us=round(us, 2), touched_experts=n_t, gbs=round(byts / us / 1e3, 1),
-            tflops=round(flops / us / 1e6, 1), hbm_frac=round(t_hbm / us, 3),
-            tc_frac=round(t_tc / us, 3), roofline_frac=round(max(t_hbm, t_tc) / us, 3),
-            bound="hbm" if t_hbm > t_tc else "tensor", includes="router + quantise + experts")
         del g
+        return dict(us=round(us, 2), touched_experts=n_t, gbs=round(byts / us / 1e3, 1),
+                    tflops=round(flops / us / 1e6, 1), hbm_frac=round(t_hbm / us, 3),
+                    tc_frac=round(t_tc / us, 3), roofline_frac=round(max(t_hbm, t_tc) / us, 3),
+                    bound="hbm" if t_hbm > t_tc else "tensor")
+
+    for T in (128, 1):
+        breakdown["fp8_dsv3_T%d" % T] = dict(fp8_entry(T, None, args.steps),
+                                             includes="router + quantise + experts")
+    # skewed sweep (Zipf 1.1 expert popularity), FP8 and the OCR-2 bf16 shape
+    sweep_steps = max(3, min(args.steps, 10))
+    sweep = {}
+    for T in (1, 8, 64, 512, 2048, 8192):
+        sweep["fp8_T%d" % T] = fp8_entry(T, 1.1, sweep_steps)
     del fp8_w
+    for T in (1, 8, 64, 512, 2048, 8192):
+        lay = inputs.ocr2_layer(T, seed=T, device=dev, weights_from=base, zipf=1.1)
+        dec = T * K <= 64
+        wsz = moe.moe_experts_workspace_size(T, H, F, E, K, 0, dec)
+        ws = torch.empty(max(wsz, 256), dtype=torch.uint8, device=dev)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        fn = moe.moe_experts_decode if dec else moe.moe_experts_prefill
+        call = lambda: fn(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K, out=out, workspace=ws)
+        t, g = time_graph(call, sweep_steps, args.warmup)
+        us = float(np.mean(t))
+        a = layer_alg(lay.idx.cpu().numpy(), T, H, F, K)
+        t_hbm = a["bytes"] / (peaks["hbm"] * 1e3)
+        t_tc = a["flops"] / (peaks["bf16"] * 1e6)
+        sweep["bf16_T%d" % T] = dict(us=round(us, 2), touched_experts=a["touched_experts"],
+                                     gbs=round(a["bytes"] / us / 1e3, 1),
+                                     tflops=round(a["flops"] / us / 1e6, 1),
+                                     roofline_frac=round(max(t_hbm, t_tc) / us, 3),
+                                     bound="hbm" if t_hbm > t_tc else "tensor")
+        del g
+    breakdown["zipf_sweep"] = sweep
 
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "decode_ocr2_T1_traffic.json")

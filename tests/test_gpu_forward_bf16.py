@@ -97,3 +97,15 @@ def test_prefill_zero_tokens_and_zero_weights(moe, cuda_dev, ocr_weights):
     lay.w.zero_()
     out = _run(moe, lay, cuda_dev, "moe_experts_prefill")
     assert torch.count_nonzero(out.float()) == 0
+
+
+@pytest.mark.parametrize("T", [64, 8192])
+def test_prefill_ocr2_zipf_sweep_sampled(moe, cuda_dev, ocr_weights, T):
+    """The OCR-2 shape of the skewed sweep: Zipf(1.1) popularity over 64 experts."""
+    lay = inputs.ocr2_layer(T, seed=11 * T, device="cpu", zipf=1.1, weights_from=ocr_weights)
+    out = _run(moe, lay, cuda_dev, "moe_experts_prefill")
+    counts = np.bincount(lay.idx.numpy().reshape(-1), minlength=64)
+    hot = int(counts.argmax())
+    rows = torch.nonzero((lay.idx == hot).any(dim=1)).reshape(-1)
+    tokens = torch.unique(torch.cat([rows[:8], torch.tensor([0, T - 1])]))
+    assert_matches_oracle(out[tokens.to(out.device)], _ref(lay, tokens), "prefill zipf T=%d" % T)

@@ -88,3 +88,21 @@ def test_fp8_dsv3_sampled(moe, cuda_dev, dsv3_weights, T):
                           "fp8 DSV3 T=%d sampled" % T)
     out2 = _run(moe, lay, idx, w, cuda_dev)
     assert torch.equal(out, out2), "fp8 path is not deterministic"
+
+
+@pytest.mark.parametrize("T", [8, 64, 2048, 8192])
+def test_fp8_dsv3_zipf_sweep_sampled(moe, cuda_dev, dsv3_weights, T):
+    """Configuration 5: Zipf(1.1) expert popularity over 256 experts; hot
+    experts get many more rows than one tile, cold experts none."""
+    lay = inputs.fp8_layer(T, seed=7 * T, device="cpu", zipf=1.1, weights=dsv3_weights)
+    idx, w = _route(lay, 8)
+    counts = np.bincount(idx.numpy().reshape(-1), minlength=256)
+    if T >= 2048:
+        assert counts.max() > 64 and (counts == 0).any()
+    out = _run(moe, lay, idx, w, cuda_dev)
+    # sample tokens routed to the hottest expert and a few others
+    hot = int(counts.argmax())
+    rows = torch.nonzero((idx == hot).any(dim=1)).reshape(-1)
+    tokens = torch.unique(torch.cat([rows[:2], torch.tensor([0, T - 1])]))[:4]
+    assert_matches_oracle(out[tokens.to(out.device)], _oracle(lay, idx, w, tokens),
+                          "fp8 DSV3 zipf T=%d sampled" % T)
