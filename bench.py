@@ -287,15 +287,16 @@ def run_ours(args):
         idx = torch.empty(T, D["K"], dtype=torch.int32, device=dev)
         tw = torch.empty(T, D["K"], dtype=torch.float32, device=dev)
         out = torch.empty(T, D["H"], dtype=torch.bfloat16, device=dev)
-        wsz = moe.moe_experts_workspace_size(T, D["H"], D["F"], D["E"], D["K"], 1, False)
+        dec = T * D["K"] <= 64
+        wsz = moe.moe_experts_workspace_size(T, D["H"], D["F"], D["E"], D["K"], 1, dec)
         ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        fn = moe.moe_experts_decode if dec else moe.moe_experts_prefill
 
         def call():
             moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"], D["topk_group"],
                                           D["K"], D["scale"], top_k_index=idx, top_k_weights=tw)
-            moe.moe_experts_prefill(lay.x, lay.w13, lay.w2, idx, tw, D["K"],
-                                    gate_up_scale=lay.w13_scale, down_scale=lay.w2_scale,
-                                    out=out, workspace=ws)
+            fn(lay.x, lay.w13, lay.w2, idx, tw, D["K"], gate_up_scale=lay.w13_scale,
+               down_scale=lay.w2_scale, out=out, workspace=ws)
         t, g = time_graph(call, steps, args.warmup)
         us = float(np.mean(t))
         n_t = len(set(idx.cpu().reshape(-1).tolist()))
@@ -309,8 +310,9 @@ def run_ours(args):
                     tc_frac=round(t_tc / us, 3), roofline_frac=round(max(t_hbm, t_tc) / us, 3),
                     bound="hbm" if t_hbm > t_tc else "tensor")
 
-    for T in (128, 1):
+    for T in (128, 8, 1):
         breakdown["fp8_dsv3_T%d" % T] = dict(fp8_entry(T, None, args.steps),
+                                             entry="decode" if T * D["K"] <= 64 else "prefill",
                                              includes="router + quantise + experts")
     # skewed sweep (Zipf 1.1 expert popularity), FP8 and the OCR-2 bf16 shape
     sweep_steps = max(3, min(args.steps, 10))
@@ -386,13 +388,17 @@ def run_only(args):
     from mixture_experts_routed_expert_b200 import inputs
 
     dev = torch.device("cuda", 0)
-    if args.only in ("fp8_128", "fp8_small"):
-        # fp8_small: the DeepSeek-V3 expert shapes with 32 experts (1.5 GB of
-        # weights) and 16 tokens, small enough for multi-pass profiler captures
+    if args.only in ("fp8_128", "fp8_small", "fp8_dec_small"):
+        # fp8_small / fp8_dec_small: the DeepSeek-V3 expert shapes with 32
+        # experts (1.5 GB of weights) and 16 tokens (prefill entry) or 1 token
+        # (decode entry), small enough for multi-pass profiler captures
         D = dict(inputs.DSV3_FP8)
         T = 128
         if args.only == "fp8_small":
             D["E"], T = 32, 16
+        if args.only == "fp8_dec_small":
+            D["E"], T = 32, 1
+        fwd = moe.moe_experts_decode if args.only == "fp8_dec_small" else moe.moe_experts_prefill
         wts = inputs.fp8_weights(seed=0, device=dev, E=D["E"])
         lay = inputs.fp8_layer(T, seed=T, device=dev, E=D["E"], weights=wts)
         flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -400,8 +406,8 @@ def run_only(args):
             flush_w.fill_(i & 0xFF)
             idx, tw = moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"],
                                                     D["topk_group"], D["K"], D["scale"])
-            out = moe.moe_experts_prefill(lay.x, lay.w13, lay.w2, idx, tw, D["K"],
-                                          gate_up_scale=lay.w13_scale, down_scale=lay.w2_scale)
+            out = fwd(lay.x, lay.w13, lay.w2, idx, tw, D["K"], gate_up_scale=lay.w13_scale,
+                      down_scale=lay.w2_scale)
         torch.cuda.synchronize()
         print("ok", args.only, float(out.float().abs().sum()))
         return
@@ -488,7 +494,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048", "fp8_128", "fp8_small"],
+    ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048", "fp8_128", "fp8_small",
+                                       "fp8_dec_small"],
                     default=None,
                     help="run just W+K eager calls of one workload (for profiler captures)")
     args = ap.parse_args()

@@ -79,8 +79,9 @@ DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t 
     L.sync = b.take(sizeof(int32_t) * decode_sync_ints(H));
     L.h = b.take(2 * N * F);
     L.ys = b.take(0);
-    L.hq = b.take(wt == MOE_W_BF16 ? 0 : N * F);
-    L.hscale = b.take(wt == MOE_W_BF16 ? 0 : sizeof(float) * N * (F / 128));
+    (void)wt;                        // the E4M3 kernels quantise h in shared memory
+    L.hq = b.take(0);
+    L.hscale = b.take(0);
     L.total = b.off;
     return L;
 }
@@ -93,6 +94,11 @@ namespace {
 
 bool decode_fits(int T, int K, int H, int F) {
     return T <= kDecodeMaxT && T * K <= kDecodeMaxSlots && decode_shape_ok(H, F);
+}
+
+// True when the decode kernels of this weight type serve T tokens.
+bool decode_serves(int T, int K, int H, int F, moe_wtype_t wt) {
+    return wt == MOE_W_FP8_E4M3 ? decode_fp8_fits(T, K, H, F) : decode_fits(T, K, H, F);
 }
 
 moe_status_t check_common(const void *x, const void *gu, const void *dn, const int32_t *idx,
@@ -159,7 +165,7 @@ const char *moe_status_string(moe_status_t s) {
 
 size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t wt, int decode) {
     if (!dims_ok(T, H, F, E, K)) return 0;
-    if (decode && decode_fits(T, K, H, F) && wt == MOE_W_BF16)
+    if (decode && (wt == MOE_W_BF16 || wt == MOE_W_FP8_E4M3) && decode_serves(T, K, H, F, wt))
         return decode_workspace(T, H, F, E, K, wt).total;
     return prefill_workspace(T, H, F, E, K, wt).total;
 }
@@ -190,14 +196,17 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
                                   out);
     if (s != MOE_OK || T == 0) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    if (!decode_fits(T, top_k, H, F) || wt != MOE_W_BF16)
+    if (!decode_serves(T, top_k, H, F, wt))
         return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                            top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
                            workspace_bytes, st);
     const DecodeWorkspace L = decode_workspace(T, H, F, E, top_k, wt);
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
         return MOE_ERR_WORKSPACE;
-    if (wt != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+    if (wt == MOE_W_FP8_E4M3)
+        return from_cuda(launch_decode_fp8(hidden_states, gate_up_proj, gate_up_scale, down_proj,
+                                           down_scale, top_k_index, top_k_weights, T, H, F, E,
+                                           top_k, static_cast<uint8_t *>(workspace), L, out, st));
     return from_cuda(launch_decode_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
                                         top_k_weights, T, H, F, E, top_k,
                                         static_cast<uint8_t *>(workspace), L, out, st));

@@ -82,6 +82,12 @@ cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *d
                                const int32_t *idx, const float *w, int T, int H, int F, int E,
                                int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
                                cudaStream_t st);
+// E4M3 decode kernels: true when T tokens x K slots fit their shared memory.
+bool decode_fp8_fits(int T, int K, int H, int F);
+cudaError_t launch_decode_fp8(const void *x, const void *w13, const float *w13s, const void *w2,
+                              const float *w2s, const int32_t *idx, const float *w, int T, int H,
+                              int F, int E, int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
+                              cudaStream_t st);
 cudaError_t launch_quantize(const void *x, int64_t rows, int cols, void *xq, float *scale,
                             cudaStream_t st);
 cudaError_t launch_route(const float *logits, const float *bias, int64_t T, int E, int num_groups,

@@ -64,12 +64,34 @@ def test_fp8_reduced_shapes(moe, cuda_dev, T, H, F, E, K, skew):
     assert_matches_oracle(out, _oracle(lay, idx, w), "fp8 T=%d H=%d F=%d E=%d" % (T, H, F, E))
 
 
-def test_fp8_decode_entry(moe, cuda_dev):
-    lay = inputs.fp8_layer(2, seed=5, device="cpu", H=512, F=256, E=32)
-    idx, w = _route(lay, 8)
-    idx[1, 3] = -1
+@pytest.mark.parametrize("T,H,F,E,K,skew", [
+    (2, 512, 256, 32, 8, None),        # two tokens, one invalid slot
+    (1, 1024, 512, 64, 8, None),       # one token: one slot per expert
+    (12, 384, 384, 4, 4, None),        # every token on all 4 experts: 12 slots each (8 + 4 ragged)
+    (16, 256, 640, 8, 4, 1.1),         # skewed: a hot expert with > 8 slots (ragged tile)
+    (5, 768, 128, 64, 6, None),        # one k-block of F, ragged token count
+])
+def test_fp8_decode_entry(moe, cuda_dev, T, H, F, E, K, skew):
+    lay = inputs.fp8_layer(T, seed=11 * T + K, device="cpu", H=H, F=F, E=E, zipf=skew)
+    idx, w = _route(lay, K, groups=min(8, E // 2), topk_group=min(4, E // 2))
+    if T >= 2:
+        idx[1, K // 2] = -1
     out = _run(moe, lay, idx, w, cuda_dev, "moe_experts_decode")
-    assert_matches_oracle(out, _oracle(lay, idx, w), "fp8 decode T=2")
+    assert_matches_oracle(out, _oracle(lay, idx, w), "fp8 decode T=%d H=%d F=%d E=%d K=%d"
+                          % (T, H, F, E, K))
+    out2 = _run(moe, lay, idx, w, cuda_dev, "moe_experts_decode")
+    assert torch.equal(out, out2), "fp8 decode is not deterministic"
+
+
+def test_fp8_decode_duplicate_and_empty(moe, cuda_dev):
+    """A token listing one expert twice (two slots, one tile column each) and a
+    token with no valid slot (its output row is zero)."""
+    lay = inputs.fp8_layer(3, seed=3, device="cpu", H=512, F=256, E=16)
+    idx = torch.tensor([[4, 4, 9, 1], [-1, 16, -1, -1], [9, 0, 4, 15]], dtype=torch.int32)
+    w = torch.rand(3, 4, generator=torch.Generator().manual_seed(0))
+    out = _run(moe, lay, idx, w, cuda_dev, "moe_experts_decode")
+    assert torch.count_nonzero(out[1]) == 0
+    assert_matches_oracle(out, _oracle(lay, idx, w), "fp8 decode duplicates")
 
 
 @pytest.fixture(scope="module")
@@ -106,3 +128,15 @@ def test_fp8_dsv3_zipf_sweep_sampled(moe, cuda_dev, dsv3_weights, T):
     tokens = torch.unique(torch.cat([rows[:2], torch.tensor([0, T - 1])]))[:4]
     assert_matches_oracle(out[tokens.to(out.device)], _oracle(lay, idx, w, tokens),
                           "fp8 DSV3 zipf T=%d sampled" % T)
+
+
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_fp8_dsv3_decode_sampled(moe, cuda_dev, dsv3_weights, T):
+    """The decode entry on the DeepSeek-V3-like layer (served by the E4M3
+    gather-GEMV kernels at these sizes)."""
+    lay = inputs.fp8_layer(T, seed=100 + T, device="cpu", weights=dsv3_weights)
+    idx, w = _route(lay, 8)
+    out = _run(moe, lay, idx, w, cuda_dev, "moe_experts_decode")
+    tokens = torch.arange(T) if T <= 4 else torch.tensor([0, 3, T - 1])
+    assert_matches_oracle(out[tokens.to(out.device)], _oracle(lay, idx, w, tokens),
+                          "fp8 DSV3 decode T=%d" % T)
