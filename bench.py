@@ -388,7 +388,7 @@ def run_only(args):
     from mixture_experts_routed_expert_b200 import inputs
 
     dev = torch.device("cuda", 0)
-    if args.only in ("fp8_128", "fp8_small", "fp8_dec_small"):
+    if args.only in ("fp8_128", "fp8_small", "fp8_dec_small", "fp8_big"):
         # fp8_small / fp8_dec_small: the DeepSeek-V3 expert shapes with 32
         # experts (1.5 GB of weights) and 16 tokens (prefill entry) or 1 token
         # (decode entry), small enough for multi-pass profiler captures
@@ -398,6 +398,9 @@ def run_only(args):
             D["E"], T = 32, 16
         if args.only == "fp8_dec_small":
             D["E"], T = 32, 1
+        if args.only == "fp8_big":
+            # 512 routed rows per expert: the tensor-bound regime on 1.4 GB of weights
+            D["E"], T = 32, 2048
         fwd = moe.moe_experts_decode if args.only == "fp8_dec_small" else moe.moe_experts_prefill
         wts = inputs.fp8_weights(seed=0, device=dev, E=D["E"])
         lay = inputs.fp8_layer(T, seed=T, device=dev, E=D["E"], weights=wts)
@@ -495,7 +498,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048", "fp8_128", "fp8_small",
-                                       "fp8_dec_small"],
+                                       "fp8_dec_small", "fp8_big"],
                     default=None,
                     help="run just W+K eager calls of one workload (for profiler captures)")
     args = ap.parse_args()

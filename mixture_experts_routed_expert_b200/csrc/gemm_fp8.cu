@@ -12,14 +12,15 @@
 //     acc[row, col] += (w_scale[row, kb] * x_scale[col, kb]) * partial[row, col]
 // while the MMA of the next k-block fills the other partial buffer.
 //   S4 (gate_up):  tile = 128 features of expert e (gate rows and up rows,
-//     two partials) x up to 64 routed rows.  h = bf16(SiLU(g) * u), then
+//     two partials) x up to BN = 64 routed rows.  h = bf16(SiLU(g) * u), then
 //     quantised per 128 features (the tile's 128 rows): scale = smallest power
 //     of two with max|h|/scale <= 448, codes E4M3 -> hq [N][F], hs [N][F/128].
-//   S5 (down):  tile = 128 hidden rows x up to 64 routed rows;
+//   S5 (down):  tile = 128 hidden rows x up to BN routed rows;
 //     y[slot, j] = w[slot] * acc  (fp32, by original slot; combined later).
 // Warp roles as in the bf16 kernel: warp 0 TMA producer, warp 1 TMEM
 // allocation + MMA issue, warps 2-9 promotion and epilogue (two warps per TMEM
-// lane quarter, each owning 32 of the 64 columns).
+// lane quarter, each owning BN/2 of the BN columns; promotion skips 16-column
+// chunks past the tile's routed rows).
 #include "common.cuh"
 #include "gemm_common.cuh"
 #include "internal.h"
@@ -28,23 +29,24 @@ namespace moe {
 
 namespace {
 
-constexpr int kBN8 = kBNFp8;          // routed rows per tile
 constexpr int kEpi8 = 8;
 constexpr int kThreads8 = 64 + 32 * kEpi8;
 constexpr int kMaxKB8 = 128;          // k-blocks (of 128) per row supported
 
-template <bool GATE_UP>
+template <bool GATE_UP, int BN>
 struct Cfg8 {
+    static_assert(BN == 64, "one epilogue thread owns 32 columns");
     static constexpr int NUM_A = GATE_UP ? 2 : 1;
     static constexpr int STAGES = GATE_UP ? 4 : 6;
     static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 e4m3
-    static constexpr int B_BYTES = kBN8 * 128;
+    static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
     static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
-    static constexpr int PCOLS = NUM_A * kBN8;          // TMEM columns of one partial buffer
-    static constexpr int TMEM_COLS = GATE_UP ? 256 : 128;
+    static constexpr int PCOLS = NUM_A * BN;            // TMEM columns of one partial buffer
+    static constexpr int TMEM_COLS = 2 * PCOLS <= 128 ? 128 : (2 * PCOLS <= 256 ? 256 : 512);  // two partial buffers, power of two
+    static constexpr int NC = BN / 2;                   // columns per epilogue thread
     static size_t smem_bytes(int E, int KB) {
-        return 1024 + RING_BYTES + 1024 + sizeof(float) * kBN8 * (KB + 1) + sizeof(float) * 5 * kBN8 +
+        return 1024 + RING_BYTES + 1024 + sizeof(float) * BN * (KB + 1) + sizeof(float) * 5 * BN +
                2 * sizeof(int) * (E + 1) + 64;
     }
 };
@@ -69,11 +71,11 @@ __device__ __forceinline__ void epi_sync() {
     asm volatile("bar.sync 2, %0;" ::"n"(32 * kEpi8) : "memory");
 }
 
-template <bool GATE_UP>
+template <bool GATE_UP, int BN>
 __global__ void __launch_bounds__(kThreads8, 1)
     grouped_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const Gemm8Args args) {
-    using C = Cfg8<GATE_UP>;
+    using C = Cfg8<GATE_UP, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,10 +86,10 @@ __global__ void __launch_bounds__(kThreads8, 1)
     uint64_t *pempty = pfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pempty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *sx = reinterpret_cast<float *>(smem + C::RING_BYTES + 1024);   // [kBN8][KB+1]
-    float *amax_s = sx + kBN8 * (args.KB + 1);                            // [4][kBN8]
-    float *scale_s = amax_s + 4 * kBN8;                                   // [kBN8]
-    int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + kBN8);
+    float *sx = reinterpret_cast<float *>(smem + C::RING_BYTES + 1024);   // [BN][KB+1]
+    float *amax_s = sx + BN * (args.KB + 1);                              // [4][BN]
+    float *scale_s = amax_s + 4 * BN;                                     // [BN]
+    int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + BN);
     int32_t *s_tiles = s_off + (args.E + 1);
     const int KB = args.KB, sxp = KB + 1;
 
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
             for (int s = 0; s < C::STAGES; ++s) armed[s] = -1;
             bool ok = true;
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, kBN8);
+                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
                 const int nbox = (t.nrows + 31) / 32;
                 const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * 32 * 128;
                 const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
@@ -168,7 +170,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
             uint32_t phase = 0, pphase = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, kBN8);
+                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
                 const uint32_t idesc = idesc_e4m3(kBM, (t.nrows + 15) & ~15);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag) ||
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         mma_e4m3_ss(d, da + 2 * k, db + 2 * k, idesc, k > 0);
-                        if (GATE_UP) mma_e4m3_ss(d + kBN8, da2 + 2 * k, db + 2 * k, idesc, k > 0);
+                        if (GATE_UP) mma_e4m3_ss(d + BN, da2 + 2 * k, db + 2 * k, idesc, k > 0);
                     }
                     mma_commit(&empty[stage]);
                     mma_commit(&pfull[pb]);
@@ -196,15 +198,16 @@ __global__ void __launch_bounds__(kThreads8, 1)
             }
         }
     } else {
+        constexpr int NC = C::NC;
         const int ew = warp - 2, et = threadIdx.x - 64;
         const int eg = warp & 3;                 // TMEM lanes [32*eg, 32*eg+32)
-        const int half = ew >> 2;                // columns [32*half, 32*half+32)
+        const int half = ew >> 2;                // columns [NC*half, NC*half+NC)
         const int row = eg * 32 + lane;
         int pb = 0;
         uint32_t pphase = 0;
         bool ok = true;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
-            const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, kBN8);
+            const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
             // activation scales of this tile's routed rows
             epi_sync();
             for (int i = et; i < t.nrows * KB; i += 32 * kEpi8) {
@@ -212,12 +215,15 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 sx[c * sxp + kb] = __ldg(args.xscale + (size_t)(t.row0 + c) * KB + kb);
             }
             epi_sync();
+            const int live = t.nrows - half * NC;   // columns of this thread that hold routed rows
             const size_t wr = (size_t)t.e * args.a_rows_per_expert + t.m * kBM + row;
             const float *wsg = args.wscale + wr * KB;
             const float *wsu = args.wscale + (wr + args.up_offset) * KB;
-            float ag[32], au[32];
+            float ag[NC], au[GATE_UP ? NC : 1];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ag[j] = au[j] = 0.f;
+            for (int j = 0; j < NC; ++j) ag[j] = 0.f;
+#pragma unroll
+            for (int j = 0; j < (GATE_UP ? NC : 1); ++j) au[j] = 0.f;
             float sg_next = __ldg(wsg), su_next = GATE_UP ? __ldg(wsu) : 0.f;
             for (int kb = 0; kb < KB; ++kb) {
                 const float sg = sg_next, su = su_next;
@@ -231,69 +237,86 @@ __global__ void __launch_bounds__(kThreads8, 1)
                     atomicOr(args.status, DEV_TIMEOUT);
                 }
                 tc_fence_after();
-                const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + pb * C::PCOLS + half * 32;
-                uint32_t pg[32], pu[32];
+                const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + pb * C::PCOLS + half * NC;
+                const float *sxk = sx + half * NC * sxp + kb;
+                // Load this thread's columns, hand the partial buffer back to
+                // the MMA warp, then promote the live 16-column chunks.
+                uint32_t pg[NC], pu[NC];
                 tmem_ld32(tb, pg);
-                if (GATE_UP) tmem_ld32(tb + kBN8, pu);
+                if (GATE_UP) tmem_ld32(tb + BN, pu);
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(&pempty[pb]);
                 if (++pb == 2) { pb = 0; pphase ^= 1; }
-                const float *sxk = sx + half * 32 * sxp + kb;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float s = sxk[j * sxp];
-                    ag[j] = fmaf(sg * s, __uint_as_float(pg[j]), ag[j]);
-                    if (GATE_UP) au[j] = fmaf(su * s, __uint_as_float(pu[j]), au[j]);
+                for (int c = 0; c < NC / 16; ++c) {
+                    if (16 * c < live) {             // warp-uniform
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float s = sxk[(16 * c + j) * sxp];
+                            ag[16 * c + j] = fmaf(sg * s, __uint_as_float(pg[16 * c + j]), ag[16 * c + j]);
+                            if (GATE_UP)
+                                au[16 * c + j] =
+                                    fmaf(su * s, __uint_as_float(pu[16 * c + j]), au[16 * c + j]);
+                        }
+                    }
                 }
             }
             if (GATE_UP) {
-                // h = bf16(SiLU(g) * u) for this row (feature) and 32 routed rows
+                // h = bf16(SiLU(g) * u) for this row (feature) and NC routed rows
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
+                for (int j = 0; j < NC; ++j)
                     ag[j] = __bfloat162float(__float2bfloat16_rn(silu_f(ag[j]) * au[j]));
-                // column max of |h| over this warp's 32 rows: lane l ends with column l
-                float v[32];
+                // column max of |h| over this warp's 32 rows, 32 columns at a
+                // time: lane l ends with column l of the group
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = fabsf(ag[j]);
+                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
+                    float v[32];
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
+                    for (int j = 0; j < 32; ++j) v[j] = 32 * grp + j < NC ? fabsf(ag[32 * grp + j]) : 0.f;
 #pragma unroll
-                    for (int i = 0; i < o; ++i) {
-                        const bool upper = (lane & o) != 0;
-                        const float send = upper ? v[i] : v[i + o];
-                        const float keep = upper ? v[i + o] : v[i];
-                        v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
+                    for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+                        for (int i = 0; i < o; ++i) {
+                            const bool upper = (lane & o) != 0;
+                            const float send = upper ? v[i] : v[i + o];
+                            const float keep = upper ? v[i + o] : v[i];
+                            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
+                        }
                     }
+                    if (32 * grp + lane < NC) amax_s[eg * BN + half * NC + 32 * grp + lane] = v[0];
                 }
-                amax_s[eg * kBN8 + half * 32 + lane] = v[0];
                 epi_sync();
-                if (et < kBN8) {
-                    const float m = fmaxf(fmaxf(amax_s[et], amax_s[kBN8 + et]),
-                                          fmaxf(amax_s[2 * kBN8 + et], amax_s[3 * kBN8 + et]));
+                if (et < BN) {
+                    const float m = fmaxf(fmaxf(amax_s[et], amax_s[BN + et]),
+                                          fmaxf(amax_s[2 * BN + et], amax_s[3 * BN + et]));
                     const int k = fp8_block_exp(m);
                     scale_s[et] = pow2f(k);
                     if (et < t.nrows) args.hs[(size_t)(t.row0 + et) * (args.F / 128) + t.m] = pow2f(k);
                 }
                 epi_sync();
-                uint8_t *hp = args.hq + (size_t)(t.row0 + half * 32) * args.F + t.m * kBM + row;
+                uint8_t *hp = args.hq + (size_t)(t.row0 + half * NC) * args.F + t.m * kBM + row;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    if (half * 32 + j < t.nrows) {
-                        const float inv = 1.0f / scale_s[half * 32 + j];
+                for (int j = 0; j < NC; ++j) {
+                    if (j < live) {
+                        const float inv = 1.0f / scale_s[half * NC + j];
                         hp[(size_t)j * args.F] = (uint8_t)(e4m3x2(ag[j] * inv, 0.f) & 0xFF);
                     }
                 }
             } else {
-                const int c = half * 32 + lane;
-                const int my_slot = (c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
-                const float my_w = (c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
                 float *yp = args.y + t.m * kBM + row;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
-                    const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
-                    if (half * 32 + j < t.nrows) yp[(size_t)slot * args.H] = wj * ag[j];
+                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
+                    const int c = half * NC + 32 * grp + lane;
+                    const int my_slot = (c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
+                    const float my_w = (c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                        const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                        if (32 * grp + j < NC && 32 * grp + j < live)
+                            yp[(size_t)slot * args.H] = wj * ag[32 * grp + j];
+                    }
                 }
             }
         }
@@ -306,25 +329,27 @@ __global__ void __launch_bounds__(kThreads8, 1)
     }
 }
 
-template <bool GATE_UP>
+template <bool GATE_UP, int BN>
 cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &b, const Gemm8Args &args,
                         cudaStream_t st) {
-    using C = Cfg8<GATE_UP>;
-    static int attr_done[64] = {};
+    using C = Cfg8<GATE_UP, BN>;
+    static size_t attr_bytes[64] = {};          // per device: dynamic shared memory limit set so far
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!attr_done[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8<GATE_UP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)C::smem_bytes(1024, kMaxKB8));
+    const size_t need = C::smem_bytes(args.E, args.KB);
+    if (need > 227 * 1024) return cudaErrorInvalidValue;
+    if (attr_bytes[dev & 63] < need) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8<GATE_UP, BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need);
         if (e != cudaSuccess) return e;
-        attr_done[dev & 63] = 1;
+        attr_bytes[dev & 63] = need;
     }
-    return launch_k(grouped_gemm_fp8<GATE_UP>, dim3(num_sms()), dim3(kThreads8),
-                    C::smem_bytes(args.E, args.KB), st, true, a, b, args);
+    return launch_k(grouped_gemm_fp8<GATE_UP, BN>, dim3(num_sms()), dim3(kThreads8), need, st, true,
+                    a, b, args);
 }
 
 }  // namespace
+
 
 cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
                              const float *topw, int64_t T, int H, int F, int E, int K, uint8_t *ws,
@@ -358,8 +383,6 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     a1.up_offset = F;
     a1.wscale = w13s;
     a1.xscale = (const float *)(ws + L.xscale);
-    cudaError_t err = launch_one8<true>(ta, tb, a1, st);
-    if (err != cudaSuccess) return err;
 
     Gemm8Args a2 = g;
     a2.tiles = (const int32_t *)(ws + L.tiles_d);
@@ -369,7 +392,9 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     a2.up_offset = 0;
     a2.wscale = w2s;
     a2.xscale = (const float *)(ws + L.hscale);
-    return launch_one8<false>(tc, td, a2, st);
+    const cudaError_t err = launch_one8<true, kBNFp8>(ta, tb, a1, st);
+    if (err != cudaSuccess) return err;
+    return launch_one8<false, kBNFp8>(tc, td, a2, st);
 }
 
 }  // namespace moe
