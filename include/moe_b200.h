@@ -119,8 +119,9 @@ MOE_API moe_status_t moe_experts_prefill(const void *hidden_states, const void *
  * Routed-experts forward, decode form: a fused gather-GEMV for a few tokens
  * (model card op "deepseek_ocr2_moe_experts_decode", n_tokens about 1-4).
  * Same arguments, layouts and results as moe_experts_prefill, workspace from
- * moe_experts_workspace_size(..., 1).  Tuned for T * K <= 64; larger calls
- * are served by the prefill kernels (same results).
+ * moe_experts_workspace_size(..., 1).  Tuned for T * K <= 64 (bf16: two
+ * gather-GEMV kernels; E4M3: the grouped GEMMs with 16-row activation
+ * tiles); larger calls are served by the prefill kernels (same results).
  */
 MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_proj,
                                 const void *down_proj, const int32_t *top_k_index,

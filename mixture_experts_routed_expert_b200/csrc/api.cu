@@ -96,10 +96,13 @@ bool decode_fits(int T, int K, int H, int F) {
     return T <= kDecodeMaxT && T * K <= kDecodeMaxSlots && decode_shape_ok(H, F);
 }
 
-// True when the decode kernels of this weight type serve T tokens.
+// True when the gather-GEMV decode kernels serve T tokens.  E4M3 weights
+// take the grouped GEMMs with 16-row activation tiles instead.
 bool decode_serves(int T, int K, int H, int F, moe_wtype_t wt) {
-    return wt == MOE_W_FP8_E4M3 ? decode_fp8_fits(T, K, H, F) : decode_fits(T, K, H, F);
+    return wt == MOE_W_BF16 && decode_fits(T, K, H, F);
 }
+// E4M3 decode-sized calls (the grouped GEMMs with 16-row tiles).
+bool fp8_decode_sized(int T, int K) { return T * K <= kDecodeMaxSlots; }
 
 moe_status_t check_common(const void *x, const void *gu, const void *dn, const int32_t *idx,
                           const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
@@ -120,16 +123,16 @@ moe_status_t check_common(const void *x, const void *gu, const void *dn, const i
 moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const int32_t *idx,
                          const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
                          const float *gus, const float *dns, void *out, void *ws, size_t ws_bytes,
-                         cudaStream_t st) {
+                         cudaStream_t st, int bn8 = kBNFp8) {
     const Workspace L = prefill_workspace(T, H, F, E, K, wt);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     const int64_t N = (int64_t)T * K;
     const bool fp8 = (wt == MOE_W_FP8_E4M3);
-    cudaError_t e = fp8 ? launch_permute_gather(x, idx, N, K, H, E, kBNFp8, kBNFp8, wt, wsb, L, st)
+    cudaError_t e = fp8 ? launch_permute_gather(x, idx, N, K, H, E, bn8, bn8, wt, wsb, L, st)
                         : launch_permute_gather(x, idx, N, K, H, E, kBNGateUp, kBNDown, wt, wsb, L, st);
     if (e == cudaSuccess)
-        e = fp8 ? launch_gemms_fp8(gu, gus, dn, dns, w, T, H, F, E, K, wsb, L, st)
+        e = fp8 ? launch_gemms_fp8(gu, gus, dn, dns, w, T, H, F, E, K, bn8, wsb, L, st)
                 : launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st);
     if (e == cudaSuccess) e = launch_combine(idx, T, H, E, K, wsb, L, out, st);
     return from_cuda(e);
@@ -199,14 +202,11 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
     if (!decode_serves(T, top_k, H, F, wt))
         return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                            top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
-                           workspace_bytes, st);
+                           workspace_bytes, st,
+                           wt == MOE_W_FP8_E4M3 && fp8_decode_sized(T, top_k) ? kBNFp8Decode : kBNFp8);
     const DecodeWorkspace L = decode_workspace(T, H, F, E, top_k, wt);
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
         return MOE_ERR_WORKSPACE;
-    if (wt == MOE_W_FP8_E4M3)
-        return from_cuda(launch_decode_fp8(hidden_states, gate_up_proj, gate_up_scale, down_proj,
-                                           down_scale, top_k_index, top_k_weights, T, H, F, E,
-                                           top_k, static_cast<uint8_t *>(workspace), L, out, st));
     return from_cuda(launch_decode_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
                                         top_k_weights, T, H, F, E, top_k,
                                         static_cast<uint8_t *>(workspace), L, out, st));

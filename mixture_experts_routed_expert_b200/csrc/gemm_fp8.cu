@@ -7,12 +7,13 @@
 // Grouped GEMM on tcgen05 with kind::f8f6f4 (E4M3 x E4M3 -> fp32, K = 32 per
 // instruction).  Because each 128-wide k-block has its own weight and
 // activation scale, every k-block's product goes to a TMEM "partial" buffer
-// (two, alternating); epilogue warps read it and promote it into fp32
+// (four in rotation; eight for 16-row tiles); epilogue warps read it and promote it into fp32
 // accumulators held in registers:
 //     acc[row, col] += (w_scale[row, kb] * x_scale[col, kb]) * partial[row, col]
 // while the MMA of the next k-block fills the other partial buffer.
 //   S4 (gate_up):  tile = 128 features of expert e (gate rows and up rows,
-//     two partials) x up to BN = 64 routed rows.  h = bf16(SiLU(g) * u), then
+//     two partials) x up to BN routed rows (64; 16 for a few tokens, where
+//     a tile per (expert, 128 features) is all there is to spread over the SMs).  h = bf16(SiLU(g) * u), then
 //     quantised per 128 features (the tile's 128 rows): scale = smallest power
 //     of two with max|h|/scale <= 448, codes E4M3 -> hq [N][F], hs [N][F/128].
 //   S5 (down):  tile = 128 hidden rows x up to BN routed rows;
@@ -35,19 +36,33 @@ constexpr int kMaxKB8 = 128;          // k-blocks (of 128) per row supported
 
 template <bool GATE_UP, int BN>
 struct Cfg8 {
-    static_assert(BN == 64, "one epilogue thread owns 32 columns");
+    static_assert(BN == 64 || BN == 16, "one epilogue thread owns 32 or 8 columns");
     static constexpr int NUM_A = GATE_UP ? 2 : 1;
-    static constexpr int STAGES = GATE_UP ? 4 : 6;
+    static constexpr int MAX_STAGES = 12;               // ring depth: chosen at launch to fill smem
+    static constexpr int BOX = BN < 32 ? BN : 32;       // routed rows per TMA box
     static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 e4m3
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
-    static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
     static constexpr int PCOLS = NUM_A * BN;            // TMEM columns of one partial buffer
-    static constexpr int TMEM_COLS = 2 * PCOLS <= 128 ? 128 : (2 * PCOLS <= 256 ? 256 : 512);  // two partial buffers, power of two
+    static constexpr int NPB = BN == 16 ? 8 : (GATE_UP ? 3 : 4);   // partial buffers in flight
+    // 64-row tiles keep their fp32 accumulators in TMEM after the partial
+    // buffers (registers would otherwise be exhausted and serialise the
+    // promotion); 16-row tiles keep them in registers.
+    static constexpr bool TACC = BN == 64;
+    static constexpr int ACC_COL = NPB * PCOLS;
+    static constexpr int COLS_USED = ACC_COL + (TACC ? NUM_A * BN : 0);
+    static constexpr int TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
+    static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
     static constexpr int NC = BN / 2;                   // columns per epilogue thread
-    static size_t smem_bytes(int E, int KB) {
-        return 1024 + RING_BYTES + 1024 + sizeof(float) * BN * (KB + 1) + sizeof(float) * 5 * BN +
-               2 * sizeof(int) * (E + 1) + 64;
+    static constexpr int CH = NC < 16 ? NC : 16;        // promotion chunk
+    // 16-row tiles (one or two per CTA) stage the weight scales in shared
+    // memory SG k-blocks ahead; wider tiles read them one k-block ahead.
+    static constexpr bool STAGE_SCALES = BN == 16;
+    static constexpr int SG = 8;                        // k-blocks per weight-scale group
+    static constexpr int WSC_FLOATS = STAGE_SCALES ? 2 * NUM_A * kBM * (SG + 1) : 0;
+    static size_t smem_bytes(int E, int KB, int stages) {
+        return 1024 + (size_t)stages * STAGE_BYTES + 1024 + sizeof(float) * WSC_FLOATS + sizeof(float) * BN * KB +
+               sizeof(float) * 5 * BN + 2 * sizeof(int) * (E + 1) + 64;
     }
 };
 
@@ -65,6 +80,7 @@ struct Gemm8Args {
     const int32_t *perm;
     const float *topw;
     int32_t *status;
+    int stages;              // depth of the TMA ring (2..MAX_STAGES)
 };
 
 __device__ __forceinline__ void epi_sync() {
@@ -80,26 +96,28 @@ __global__ void __launch_bounds__(kThreads8, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *ring = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::RING_BYTES);
-    uint64_t *empty = full + C::STAGES;
-    uint64_t *pfull = empty + C::STAGES;
-    uint64_t *pempty = pfull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pempty + 2);
+    const int NST = args.stages;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)NST * C::STAGE_BYTES);
+    uint64_t *empty = full + C::MAX_STAGES;
+    uint64_t *pfull = empty + C::MAX_STAGES;
+    uint64_t *pempty = pfull + C::NPB;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pempty + C::NPB);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *sx = reinterpret_cast<float *>(smem + C::RING_BYTES + 1024);   // [BN][KB+1]
-    float *amax_s = sx + BN * (args.KB + 1);                              // [4][BN]
+    float *wsc = reinterpret_cast<float *>(smem + (size_t)NST * C::STAGE_BYTES + 1024);  // [2][NUM_A][128][SG+1]
+    float *sx = wsc + C::WSC_FLOATS;                                      // [KB][BN]
+    float *amax_s = sx + BN * args.KB;                                    // [4][BN]
     float *scale_s = amax_s + 4 * BN;                                     // [BN]
     int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + BN);
     int32_t *s_tiles = s_off + (args.E + 1);
-    const int KB = args.KB, sxp = KB + 1;
+    const int KB = args.KB;
 
     const int warp = threadIdx.x >> 5, lane = lane_id();
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::NPB; ++b) {
             mbar_init(&pfull[b], 1);
             mbar_init(&pempty[b], 32 * kEpi8);
         }
@@ -130,14 +148,14 @@ __global__ void __launch_bounds__(kThreads8, 1)
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_x = policy_evict_last();
-            int stage = 0, armed[C::STAGES];
+            int stage = 0, armed[C::MAX_STAGES];
             uint32_t phase = 0;
-            for (int s = 0; s < C::STAGES; ++s) armed[s] = -1;
+            for (int s = 0; s < C::MAX_STAGES; ++s) armed[s] = -1;
             bool ok = true;
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
-                const int nbox = (t.nrows + 31) / 32;
-                const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * 32 * 128;
+                const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
+                const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * C::BOX * 128;
                 const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
@@ -150,9 +168,9 @@ __global__ void __launch_bounds__(kThreads8, 1)
                         tma_load_2d(sA + C::A_BYTES, &tmA, &full[stage], kb * 128,
                                     arow + args.up_offset, pol_w);
                     for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sB + b * 32 * 128, &tmB, &full[stage], kb * 128,
-                                    t.row0 + b * 32, pol_x);
-                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+                        tma_load_2d(sB + b * C::BOX * 128, &tmB, &full[stage], kb * 128,
+                                    t.row0 + b * C::BOX, pol_x);
+                    if (++stage == NST) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok) {
@@ -160,7 +178,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 atomicOr(args.status, DEV_TIMEOUT);
             }
             volatile int never = 0;
-            for (int s = 0; s < C::STAGES; ++s)
+            for (int s = 0; s < NST; ++s)
                 if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
                     atomicOr(args.status, DEV_TIMEOUT);
         }
@@ -188,8 +206,8 @@ __global__ void __launch_bounds__(kThreads8, 1)
                     }
                     mma_commit(&empty[stage]);
                     mma_commit(&pfull[pb]);
-                    if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-                    if (++pb == 2) { pb = 0; pphase ^= 1; }
+                    if (++stage == NST) { stage = 0; phase ^= 1; }
+                    if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
                 }
             }
             if (!ok) {
@@ -212,24 +230,60 @@ __global__ void __launch_bounds__(kThreads8, 1)
             epi_sync();
             for (int i = et; i < t.nrows * KB; i += 32 * kEpi8) {
                 const int c = i / KB, kb = i - c * KB;
-                sx[c * sxp + kb] = __ldg(args.xscale + (size_t)(t.row0 + c) * KB + kb);
+                sx[kb * BN + c] = __ldg(args.xscale + (size_t)(t.row0 + c) * KB + kb);
             }
             epi_sync();
             const int live = t.nrows - half * NC;   // columns of this thread that hold routed rows
-            const size_t wr = (size_t)t.e * args.a_rows_per_expert + t.m * kBM + row;
-            const float *wsg = args.wscale + wr * KB;
-            const float *wsu = args.wscale + (wr + args.up_offset) * KB;
+            // Weight scales of the tile's 128 rows: with STAGE_SCALES they
+            // arrive in shared memory SG k-blocks at a time, one group ahead
+            // (asynchronous copies); otherwise each is read one k-block ahead.
+            const float *wsrc = args.wscale + ((size_t)t.e * args.a_rows_per_expert + t.m * kBM) * KB;
+            const float *wsg = wsrc + (size_t)row * KB;
+            const float *wsu = wsrc + (size_t)(row + args.up_offset) * KB;
+            auto issue_scales = [&](int kb0, int buf) {
+                for (int i = et; i < C::NUM_A * kBM * C::SG; i += 32 * kEpi8) {
+                    const int a = i / (kBM * C::SG), r = (i / C::SG) % kBM, q = i % C::SG;
+                    if (kb0 + q < KB)
+                        cp_async4(wsc + ((buf * C::NUM_A + a) * kBM + r) * (C::SG + 1) + q,
+                                  wsrc + (size_t)(a * args.up_offset + r) * KB + kb0 + q);
+                }
+                cp_async_commit();
+            };
             float ag[NC], au[GATE_UP ? NC : 1];
 #pragma unroll
             for (int j = 0; j < NC; ++j) ag[j] = 0.f;
 #pragma unroll
             for (int j = 0; j < (GATE_UP ? NC : 1); ++j) au[j] = 0.f;
-            float sg_next = __ldg(wsg), su_next = GATE_UP ? __ldg(wsu) : 0.f;
+            float sg_next = 0.f, su_next = 0.f;
+            if constexpr (C::STAGE_SCALES) {
+                issue_scales(0, 0);
+            } else {
+                sg_next = __ldg(wsg);
+                if (GATE_UP) su_next = __ldg(wsu);
+            }
             for (int kb = 0; kb < KB; ++kb) {
-                const float sg = sg_next, su = su_next;
-                if (kb + 1 < KB) {
-                    sg_next = __ldg(wsg + kb + 1);
-                    if (GATE_UP) su_next = __ldg(wsu + kb + 1);
+                const int grp = kb / C::SG, q = kb - grp * C::SG, buf = grp & 1;
+                float sg, su;
+                if constexpr (!C::STAGE_SCALES) {
+                    sg = sg_next;
+                    su = su_next;
+                    if (kb + 1 < KB) {
+                        sg_next = __ldg(wsg + kb + 1);
+                        if (GATE_UP) su_next = __ldg(wsu + kb + 1);
+                    }
+                } else {
+                    if (q == 0) {
+                        epi_sync();                  // everyone is done with the other buffer
+                        if (kb + C::SG < KB) {
+                            issue_scales(kb + C::SG, buf ^ 1);
+                            cp_async_wait<1>();
+                        } else {
+                            cp_async_wait<0>();
+                        }
+                        epi_sync();                  // this group's scales are visible
+                    }
+                    sg = wsc[((buf * C::NUM_A) * kBM + row) * (C::SG + 1) + q];
+                    su = GATE_UP ? wsc[((buf * C::NUM_A + 1) * kBM + row) * (C::SG + 1) + q] : 0.f;
                 }
                 if (ok && !mbar_wait(&pfull[pb], pphase, abort_flag)) {
                     ok = false;
@@ -238,28 +292,95 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 }
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + pb * C::PCOLS + half * NC;
-                const float *sxk = sx + half * NC * sxp + kb;
+                const uint32_t tacc = tmem_base + ((uint32_t)(eg * 32) << 16) + C::ACC_COL + half * NC;
+                const float *sxk = sx + kb * BN + half * NC;   // this thread's column scales
                 // Load this thread's columns, hand the partial buffer back to
                 // the MMA warp, then promote the live 16-column chunks.
                 uint32_t pg[NC], pu[NC];
-                tmem_ld32(tb, pg);
-                if (GATE_UP) tmem_ld32(tb + BN, pu);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&pempty[pb]);
-                if (++pb == 2) { pb = 0; pphase ^= 1; }
+                auto promote = [&](int c) {          // chunk c of C::CH columns
+                    if (C::CH * c < live) {          // warp-uniform
 #pragma unroll
-                for (int c = 0; c < NC / 16; ++c) {
-                    if (16 * c < live) {             // warp-uniform
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const float s = sxk[(16 * c + j) * sxp];
-                            ag[16 * c + j] = fmaf(sg * s, __uint_as_float(pg[16 * c + j]), ag[16 * c + j]);
-                            if (GATE_UP)
-                                au[16 * c + j] =
-                                    fmaf(su * s, __uint_as_float(pu[16 * c + j]), au[16 * c + j]);
+                        for (int j = 0; j < C::CH; ++j) {
+                            const int q = C::CH * c + j;
+                            const float s = sxk[q];
+                            ag[q] = fmaf(sg * s, __uint_as_float(pg[q]), ag[q]);
+                            if (GATE_UP) au[q] = fmaf(su * s, __uint_as_float(pu[q]), au[q]);
                         }
                     }
+                };
+                if constexpr (C::TACC) {
+                    // partials of both halves, then the buffer goes back to the
+                    // MMA warp; accumulators: TMEM -> registers -> TMEM
+                    tmem_ld32(tb, pg);
+                    if (GATE_UP) tmem_ld32(tb + BN, pu);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&pempty[pb]);
+                    if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (16 * h < live) {         // warp-uniform
+                            uint32_t a_g[16], a_u[16];
+                            if (kb > 0) {
+                                tmem_ld16(tacc + 16 * h, a_g);
+                                if (GATE_UP) tmem_ld16(tacc + BN + 16 * h, a_u);
+                                tmem_ld_wait_regs16(a_g);
+                                if (GATE_UP) tmem_ld_wait_regs16(a_u);
+                            }
+                            // pairs of columns: (w_scale * x_scale) and the fma
+                            // on fp32x2, the same roundings as the scalar form
+                            const float2 sg2 = make_float2(sg, sg), su2 = make_float2(su, su);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float4 s4 = *reinterpret_cast<const float4 *>(sxk + 16 * h + 4 * i);
+#pragma unroll
+                                for (int k = 0; k < 2; ++k) {
+                                    const int j = 4 * i + 2 * k, q = 16 * h + j;
+                                    const float2 sc = k == 0 ? make_float2(s4.x, s4.y) : make_float2(s4.z, s4.w);
+                                    const float2 p2 = make_float2(__uint_as_float(pg[q]), __uint_as_float(pg[q + 1]));
+                                    const float2 a2 = kb > 0 ? make_float2(__uint_as_float(a_g[j]), __uint_as_float(a_g[j + 1]))
+                                                             : make_float2(0.f, 0.f);
+                                    const float2 r2 = __ffma2_rn(__fmul2_rn(sg2, sc), p2, a2);
+                                    a_g[j] = __float_as_uint(r2.x);
+                                    a_g[j + 1] = __float_as_uint(r2.y);
+                                    if (GATE_UP) {
+                                        const float2 pu2 = make_float2(__uint_as_float(pu[q]), __uint_as_float(pu[q + 1]));
+                                        const float2 b2 = kb > 0 ? make_float2(__uint_as_float(a_u[j]), __uint_as_float(a_u[j + 1]))
+                                                                 : make_float2(0.f, 0.f);
+                                        const float2 t2 = __ffma2_rn(__fmul2_rn(su2, sc), pu2, b2);
+                                        a_u[j] = __float_as_uint(t2.x);
+                                        a_u[j + 1] = __float_as_uint(t2.y);
+                                    }
+                                }
+                            }
+                            tmem_st16(tacc + 16 * h, a_g);
+                            if (GATE_UP) tmem_st16(tacc + BN + 16 * h, a_u);
+                        }
+                    }
+                    tmem_st_wait();
+                } else {
+                    tmem_ld8(tb, pg);
+                    if (GATE_UP) tmem_ld8(tb + BN, pu);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&pempty[pb]);
+                    if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
+#pragma unroll
+                    for (int c = 0; c < NC / C::CH; ++c) promote(c);
+                }
+            }
+            if constexpr (C::TACC) {
+                const uint32_t tacc = tmem_base + ((uint32_t)(eg * 32) << 16) + C::ACC_COL + half * NC;
+                uint32_t r[NC];
+                tmem_ld32(tacc, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < NC; ++j) ag[j] = __uint_as_float(r[j]);
+                if (GATE_UP) {
+                    tmem_ld32(tacc + BN, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < NC; ++j) au[j] = __uint_as_float(r[j]);
                 }
             }
             if (GATE_UP) {
@@ -336,8 +457,12 @@ cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &b, const Gemm8A
     static size_t attr_bytes[64] = {};          // per device: dynamic shared memory limit set so far
     int dev = 0;
     cudaGetDevice(&dev);
-    const size_t need = C::smem_bytes(args.E, args.KB);
-    if (need > 227 * 1024) return cudaErrorInvalidValue;
+    constexpr size_t kSmemMax = 227 * 1024;
+    Gemm8Args a8 = args;
+    a8.stages = C::MAX_STAGES;
+    while (a8.stages > 2 && C::smem_bytes(args.E, args.KB, a8.stages) > kSmemMax) --a8.stages;
+    const size_t need = C::smem_bytes(args.E, args.KB, a8.stages);
+    if (need > kSmemMax) return cudaErrorInvalidValue;
     if (attr_bytes[dev & 63] < need) {
         cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8<GATE_UP, BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need);
@@ -345,23 +470,25 @@ cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &b, const Gemm8A
         attr_bytes[dev & 63] = need;
     }
     return launch_k(grouped_gemm_fp8<GATE_UP, BN>, dim3(num_sms()), dim3(kThreads8), need, st, true,
-                    a, b, args);
+                    a, b, a8);
 }
 
 }  // namespace
 
 
 cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
-                             const float *topw, int64_t T, int H, int F, int E, int K, uint8_t *ws,
-                             const Workspace &L, cudaStream_t st) {
+                             const float *topw, int64_t T, int H, int F, int E, int K, int bn,
+                             uint8_t *ws, const Workspace &L, cudaStream_t st) {
     if (H / 128 > kMaxKB8 || F / 128 > kMaxKB8) return cudaErrorInvalidValue;
+    if (bn != kBNFp8 && bn != kBNFp8Decode) return cudaErrorInvalidValue;
+    const int box = bn < 32 ? bn : 32;
     const uint64_t N = (uint64_t)T * K;
     CUtensorMap ta, tb, tc, td;
     const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
     if (!make_tmap(&ta, U8, 1, w13, (uint64_t)E * 2 * F, H, kBM) ||
-        !make_tmap(&tb, U8, 1, ws + L.xperm, N, H, 32) ||
+        !make_tmap(&tb, U8, 1, ws + L.xperm, N, H, box) ||
         !make_tmap(&tc, U8, 1, w2, (uint64_t)E * H, F, kBM) ||
-        !make_tmap(&td, U8, 1, ws + L.h, N, F, 32))
+        !make_tmap(&td, U8, 1, ws + L.h, N, F, box))
         return cudaErrorInvalidValue;
     Gemm8Args g = {};
     g.offsets = (const int32_t *)(ws + L.offsets);
@@ -392,6 +519,11 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     a2.up_offset = 0;
     a2.wscale = w2s;
     a2.xscale = (const float *)(ws + L.hscale);
+    if (bn == kBNFp8Decode) {
+        const cudaError_t err = launch_one8<true, kBNFp8Decode>(ta, tb, a1, st);
+        if (err != cudaSuccess) return err;
+        return launch_one8<false, kBNFp8Decode>(tc, td, a2, st);
+    }
     const cudaError_t err = launch_one8<true, kBNFp8>(ta, tb, a1, st);
     if (err != cudaSuccess) return err;
     return launch_one8<false, kBNFp8>(tc, td, a2, st);

@@ -16,6 +16,7 @@ constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBNGateUp = 128;    // routed rows (tokens) per gate_up tile
 constexpr int kBNDown = 256;      // routed rows per down tile
 constexpr int kBNFp8 = 64;        // routed rows per tile of both E4M3 GEMMs
+constexpr int kBNFp8Decode = 16;  // the same GEMMs for a few tokens (decode entry)
 
 // ---- workspace layout ------------------------------------------------------
 struct Workspace {
@@ -73,21 +74,16 @@ cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, con
 cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float *topw, int64_t T,
                               int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
                               cudaStream_t st);
+// bn: kBNFp8 or kBNFp8Decode; must match the tile prefixes of the permutation.
 cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
-                             const float *topw, int64_t T, int H, int F, int E, int K, uint8_t *ws,
-                             const Workspace &L, cudaStream_t st);
+                             const float *topw, int64_t T, int H, int F, int E, int K, int bn,
+                             uint8_t *ws, const Workspace &L, cudaStream_t st);
 cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, const uint8_t *ws,
                            const Workspace &L, void *out, cudaStream_t st);
 cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *down,
                                const int32_t *idx, const float *w, int T, int H, int F, int E,
                                int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
                                cudaStream_t st);
-// E4M3 decode kernels: true when T tokens x K slots fit their shared memory.
-bool decode_fp8_fits(int T, int K, int H, int F);
-cudaError_t launch_decode_fp8(const void *x, const void *w13, const float *w13s, const void *w2,
-                              const float *w2s, const int32_t *idx, const float *w, int T, int H,
-                              int F, int E, int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
-                              cudaStream_t st);
 cudaError_t launch_quantize(const void *x, int64_t rows, int cols, void *xq, float *scale,
                             cudaStream_t st);
 cudaError_t launch_route(const float *logits, const float *bias, int64_t T, int E, int num_groups,

@@ -15,6 +15,8 @@
 // recounts the whole routing (T*K int32, read from L2) to get the expert
 // offsets and the number of earlier slots of each expert before its own chunk,
 // ranks its chunk's slots stably, writes perm / inv and gathers its rows.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -66,7 +68,10 @@ __device__ int block_scan_inplace(int32_t *v, int n) {
 
 // MODE 0: permutation only; 1: + bf16 row gather; 2: + gather with block-128
 // E4M3 quantisation (the rule of quantize_fp8_block128).
-// Block b handles slots [b*chunk, (b+1)*chunk), chunk <= kPThreads.
+// Block (b, c) handles slots [b*chunk, (b+1)*chunk), chunk <= kPThreads, and
+// gathers column slice c of their rows (gridDim.y slices of whole 128-column
+// blocks, so that a few slots still spread over many blocks); only blocks
+// with c = 0 write the permutation.
 // Dynamic shared memory: cnt_all[E+1], cnt_before[E], wc[kPWarps][E], tiles[E+1].
 template <int MODE>
 __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
@@ -117,7 +122,8 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
         }
     }
     __syncthreads();
-    if (blockIdx.x == 0)
+    const bool lead = blockIdx.x == 0 && blockIdx.y == 0;   // writes counts, offsets, tiles
+    if (lead)
         for (int i = t; i < E; i += kPThreads) {
             counts[i] = cnt_all[i];
             tl[i] = cnt_all[i];
@@ -137,11 +143,11 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
         int r = rank_w;
         for (int w = 0; w < warp; ++w) r += wc[w * E + e];
         pos = cnt_all[e] + cnt_bef[e] + r;
-        perm[pos] = s;
+        if (blockIdx.y == 0) perm[pos] = s;
     }
-    if (mine) inv[s] = pos;
+    if (mine && blockIdx.y == 0) inv[s] = pos;
     pos_s[t] = mine ? pos : -1;
-    if (blockIdx.x == 0) {
+    if (lead) {
         if (t == 0) {
             *status = 0;
             offsets[E] = total;
@@ -164,20 +170,24 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
     }
     __syncthreads();
     if (MODE == 0) return;
-    // 3. gather the chunk's rows: one warp per row, 16-byte vectors
+    // 3. gather the chunk's rows (this block's column slice): one warp per
+    //    row, 16-byte vectors
     const int nv = H / 8;
+    const int nb16 = (nv + 15) / 16;                       // 128-column blocks
+    const int vs0 = 16 * (int)((int64_t)nb16 * blockIdx.y / gridDim.y);
+    const int vs1 = min(nv, 16 * (int)((int64_t)nb16 * (blockIdx.y + 1) / gridDim.y));
     for (int r = warp; r < chunk; r += kPWarps) {
         const int p = pos_s[r];
         if (p < 0) continue;
         const uint4 *src = x + (size_t)((c0 + r) / K) * nv;
         if (MODE == 1) {
             uint4 *dst = reinterpret_cast<uint4 *>(xperm) + (size_t)p * nv;
-            for (int v = lane; v < nv; v += 32) dst[v] = __ldg(src + v);
+            for (int v = vs0 + lane; v < vs1; v += 32) dst[v] = __ldg(src + v);
         } else {
             uint2 *dst = reinterpret_cast<uint2 *>(xperm) + (size_t)p * nv;
-            for (int v0 = 0; v0 < nv; v0 += 32) {
+            for (int v0 = vs0; v0 < vs1; v0 += 32) {
                 const int v = v0 + lane;
-                const bool on = v < nv;
+                const bool on = v < vs1;
                 float f[8];
                 unpack_bf16x8(on ? __ldg(src + v) : make_uint4(0, 0, 0, 0), f);
                 float sc;
@@ -202,12 +212,25 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
     if (i >= T * nv) return;
     const int64_t t = i / nv;
     const int v = (int)(i - t * nv);
+    // ids first (one mask), then every row load at once, then the sum in k order
+    unsigned valid = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        if (k < K) {
+            const int e = __ldg(idx + t * K + k);
+            if (e >= 0 && e < E) valid |= 1u << k;
+        }
+    }
+    float4 a[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+        a[k] = (valid >> k) & 1u ? __ldcs(y + (t * K + k) * nv + v) : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < K; ++k) {
-        const int e = __ldg(idx + t * K + k);
-        if (e < 0 || e >= E) continue;
-        const float4 a = __ldcs(y + (t * K + k) * nv + v);
-        acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        if ((valid >> k) & 1u) {
+            acc.x += a[k].x; acc.y += a[k].y; acc.z += a[k].z; acc.w += a[k].w;
+        }
     }
     uint2 o;
     o.x = pack_bf16x2(acc.x, acc.y);
@@ -235,7 +258,12 @@ cudaError_t launch_pg(const void *x, const int32_t *idx, int64_t n_slots, int K,
     const int64_t floor_chunk = n_slots > 32768 ? 128 : 8;
     while (chunk > floor_chunk && n_slots / chunk < 2 * num_sms()) chunk /= 2;
     const unsigned blocks = (unsigned)((n_slots + chunk - 1) / chunk);
-    return launch_k(permute_gather_kernel<MODE>, dim3(blocks), dim3(kPThreads), smem, st, false,
+    // column slices: enough blocks for about two per SM when there are few slots
+    const int nb16 = (H / 8 + 15) / 16;
+    const unsigned slices = MODE == 0 ? 1u
+                                      : (unsigned)std::max<int64_t>(
+                                            1, std::min<int64_t>(nb16, (2 * num_sms() + blocks - 1) / blocks));
+    return launch_k(permute_gather_kernel<MODE>, dim3(blocks, slices), dim3(kPThreads), smem, st, false,
                     idx, (int)n_slots, E, K, H, chunk, bn_g, bn_d, (const uint4 *)x,
                     (void *)(ws + L.xperm), (float *)(ws + L.xscale), (int32_t *)(ws + L.counts),
                     (int32_t *)(ws + L.offsets), (int32_t *)(ws + L.tiles_g),
