@@ -25,84 +25,105 @@ __global__ void __launch_bounds__(256) quantize_kernel(const uint4 *__restrict__
     }
 }
 
-constexpr int kRouteWarps = 4;
+constexpr int kRouteThreads = 256;
 
 // "a ranks before b": larger score first, lower index on equal scores.
 __device__ __forceinline__ bool ranks_before(float sa, int ia, float sb, int ib) {
     return sa > sb || (sa == sb && ia < ib);
 }
 
-// One warp per token.  smem per warp: s[E] and c[E].
-__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(
+// Best two of a group held as (value, index) pairs: merge (b1, b2) into (a1, a2).
+__device__ __forceinline__ void top2_merge(float &a1, int &i1, float &a2, int &j2, float b1, int k1,
+                                           float b2, int k2) {
+    if (k1 >= 0 && (i1 < 0 || ranks_before(b1, k1, a1, i1))) {
+        // b1 is the new best; the second is the better of a1 and b1's partner
+        if (i1 >= 0 && (k2 < 0 || ranks_before(a1, i1, b2, k2))) { a2 = a1; j2 = i1; }
+        else { a2 = b2; j2 = k2; }
+        a1 = b1; i1 = k1;
+    } else if (k1 >= 0 && (j2 < 0 || ranks_before(b1, k1, a2, j2))) {
+        a2 = b1; j2 = k1;
+    }
+}
+
+// One block per token.  s[e] = sigmoid(logit) (double, rounded to fp32),
+// c[e] = s[e] + bias[e] (selection score).  Groups are scored by the sum of
+// their two best c, the topk_group best groups are kept, and the top_k
+// experts of the kept groups are chosen; every selection uses the order
+// (score desc, index asc), so each candidate's position is the number of
+// candidates ranking before it.  Weights: s of the chosen experts divided by
+// their sum (summed in choice order), times the scaling factor.
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(
     const float *__restrict__ logits, const float *__restrict__ bias, int64_t T, int E, int G,
     int topk_group, int top_k, float scale, int32_t *__restrict__ idx, float *__restrict__ wout) {
     extern __shared__ float rsm[];
-    const int warp = threadIdx.x >> 5, lane = lane_id();
-    const int64_t t = (int64_t)blockIdx.x * kRouteWarps + warp;
-    if (t >= T) return;
-    float *s = rsm + (size_t)warp * 2 * E;
-    float *c = s + E;
-    for (int e = lane; e < E; e += 32) {
+    float *s = rsm;              // [E]
+    float *c = s + E;            // [E]
+    __shared__ float gsc[32];
+    __shared__ unsigned keep_s;
+    __shared__ float sel_s[16];
+    __shared__ float sum_s;
+    const int64_t t = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = lane_id();
+    for (int e = tid; e < E; e += kRouteThreads) {
         const double lg = (double)__ldg(logits + t * E + e);
         const float se = (float)(1.0 / (1.0 + exp(-lg)));
         s[e] = se;
         c[e] = se + __ldg(bias + e);
     }
-    __syncwarp();
-    // group scores: sum of the two best c in each group (lane g owns group g)
+    __syncthreads();
+    // group scores: one warp per group (lanes stride over the group)
     const int gsize = E / G;
-    float gs = -INFINITY;
-    if (lane < G) {
-        int b1 = -1, b2 = -1;
-        for (int e = lane * gsize; e < (lane + 1) * gsize; ++e) {
-            if (b1 < 0 || ranks_before(c[e], e, c[b1], b1)) { b2 = b1; b1 = e; }
-            else if (b2 < 0 || ranks_before(c[e], e, c[b2], b2)) { b2 = e; }
-        }
-        gs = (b2 >= 0) ? c[b1] + c[b2] : c[b1];
-    }
-    // keep the topk_group best groups
-    unsigned keep = 0;
-    for (int r = 0; r < topk_group; ++r) {
-        float bv = (lane < G && !((keep >> lane) & 1u)) ? gs : -INFINITY;
-        int bi = (lane < G && !((keep >> lane) & 1u)) ? lane : 0x7FFFFFFF;
+    for (int g = warp; g < G; g += kRouteThreads / 32) {
+        float a1 = 0.f, a2 = 0.f;
+        int i1 = -1, j2 = -1;
+        for (int e = g * gsize + lane; e < (g + 1) * gsize; e += 32) top2_merge(a1, i1, a2, j2, c[e], e, 0.f, -1);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
-            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-            if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ranks_before(ov, oi, bv, bi))) { bv = ov; bi = oi; }
+            const float b1 = __shfl_xor_sync(0xFFFFFFFFu, a1, o), b2 = __shfl_xor_sync(0xFFFFFFFFu, a2, o);
+            const int k1 = __shfl_xor_sync(0xFFFFFFFFu, i1, o), k2 = __shfl_xor_sync(0xFFFFFFFFu, j2, o);
+            top2_merge(a1, i1, a2, j2, b1, k1, b2, k2);
         }
-        keep |= 1u << bi;
+        if (lane == 0) gsc[g] = (j2 >= 0) ? c[i1] + c[j2] : c[i1];
     }
-    // top_k experts among the kept groups
-    unsigned taken = 0;  // bit i: expert lane + 32 i already chosen
-    int chosen = -1;     // lane k keeps the k-th choice
-    for (int k = 0; k < top_k; ++k) {
-        float bv = -INFINITY;
-        int bi = 0x7FFFFFFF;
-        for (int i = 0, e = lane; e < E; ++i, e += 32) {
-            if (((keep >> (e / gsize)) & 1u) && !((taken >> i) & 1u) &&
-                (bi == 0x7FFFFFFF || ranks_before(c[e], e, bv, bi))) {
-                bv = c[e];
-                bi = e;
-            }
+    __syncthreads();
+    // kept groups: rank of each group score among all G
+    if (warp == 0) {
+        bool kept = false;
+        if (lane < G) {
+            const float v = gsc[lane];
+            int r = 0;
+            for (int g = 0; g < G; ++g) r += ranks_before(gsc[g], g, v, lane);
+            kept = r < topk_group;
         }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
-            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-            if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ranks_before(ov, oi, bv, bi))) { bv = ov; bi = oi; }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (lane == k) chosen = bi;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, kept);
+        if (lane == 0) keep_s = m;
     }
-    // weights: unbiased scores normalised over the choices, in choice order
-    const float sk = (lane < top_k) ? s[chosen] : 0.f;
-    float sum = 0.f;
-    for (int k = 0; k < top_k; ++k) sum += __shfl_sync(0xFFFFFFFFu, sk, k);
-    if (lane < top_k) {
-        const float q = sk / sum;
-        idx[t * top_k + lane] = chosen;
-        wout[t * top_k + lane] = q * scale;
+    __syncthreads();
+    const unsigned keep = keep_s;
+    // chosen experts: rank of each kept candidate among the kept candidates
+    for (int e = tid; e < E; e += kRouteThreads) {
+        if (!((keep >> (e / gsize)) & 1u)) continue;
+        const float v = c[e];
+        int r = 0;
+        for (int g = 0; g < G; ++g) {
+            if (!((keep >> g) & 1u)) continue;
+            for (int q = g * gsize; q < (g + 1) * gsize; ++q) r += ranks_before(c[q], q, v, e);
+        }
+        if (r < top_k) {
+            idx[t * top_k + r] = e;
+            sel_s[r] = s[e];
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float sum = 0.f;
+        for (int k = 0; k < top_k; ++k) sum += sel_s[k];
+        sum_s = sum;
+    }
+    __syncthreads();
+    if (tid < top_k) {
+        const float q = sel_s[tid] / sum_s;
+        wout[t * top_k + tid] = q * scale;
     }
 }
 
@@ -159,19 +180,9 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int cols, void *xq, flo
 cudaError_t launch_route(const float *logits, const float *bias, int64_t T, int E, int num_groups,
                          int topk_group, int top_k, float scale, int32_t *idx, float *w,
                          int32_t *offsets, cudaStream_t st) {
-    const size_t smem = sizeof(float) * 2 * E * kRouteWarps;
-    static int attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!attr_done[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(sizeof(float) * 2 * 1024 * kRouteWarps));
-        if (e != cudaSuccess) return e;
-        attr_done[dev & 63] = 1;
-    }
-    cudaError_t err = launch_k(route_kernel, dim3((unsigned)((T + kRouteWarps - 1) / kRouteWarps)),
-                               dim3(kRouteWarps * 32), smem, st, false, logits, bias, T, E,
-                               num_groups, topk_group, top_k, scale, idx, w);
+    const size_t smem = sizeof(float) * 2 * E;            // <= 8 KB for E <= 1024
+    cudaError_t err = launch_k(route_kernel, dim3((unsigned)T), dim3(kRouteThreads), smem, st, false,
+                               logits, bias, T, E, num_groups, topk_group, top_k, scale, idx, w);
     if (err != cudaSuccess || offsets == nullptr) return err;
     return launch_k(route_offsets_kernel, dim3(1), dim3(1024), 0, st, true, (const int32_t *)idx,
                     T * top_k, E, offsets);
