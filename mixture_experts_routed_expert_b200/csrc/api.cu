@@ -96,10 +96,14 @@ bool decode_fits(int T, int K, int H, int F) {
     return T <= kDecodeMaxT && T * K <= kDecodeMaxSlots && decode_shape_ok(H, F);
 }
 
-// True when the gather-GEMV decode kernels serve T tokens.  E4M3 weights
-// take the grouped GEMMs with 16-row activation tiles instead.
+// True when the gather-GEMV decode kernels serve T tokens: bf16 weights and
+// at most kGemvMaxSlots slots (beyond that the grouped GEMMs, which stream
+// each touched expert once through TMA, are faster: OCR-2 shape T=4 / 8 ->
+// 47 / 64 us against 51 / 90 us).  E4M3 weights take the grouped GEMMs with
+// 16-row activation tiles instead.
+constexpr int kGemvMaxSlots = 16;
 bool decode_serves(int T, int K, int H, int F, moe_wtype_t wt) {
-    return wt == MOE_W_BF16 && decode_fits(T, K, H, F);
+    return wt == MOE_W_BF16 && T * K <= kGemvMaxSlots && decode_fits(T, K, H, F);
 }
 // E4M3 decode-sized calls (the grouped GEMMs with 16-row tiles).
 bool fp8_decode_sized(int T, int K) { return T * K <= kDecodeMaxSlots; }
