@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
     if (i >= T * nv) return;
     const int64_t t = i / nv;
     const int v = (int)(i - t * nv);
-    // ids first (one mask), then every row load at once, then the sum in k order
+    // ids first (one mask), then the row loads four at a time, summed in k order
     unsigned valid = 0;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -221,15 +221,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
             if (e >= 0 && e < E) valid |= 1u << k;
         }
     }
-    float4 a[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-        a[k] = (valid >> k) & 1u ? __ldcs(y + (t * K + k) * nv + v) : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = 0; k0 < K; k0 += 4) {       // four row loads in flight, then their sum
+        float4 a[4];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        if ((valid >> k) & 1u) {
-            acc.x += a[k].x; acc.y += a[k].y; acc.z += a[k].z; acc.w += a[k].w;
+        for (int i = 0; i < 4; ++i)
+            a[i] = (valid >> (k0 + i)) & 1u ? __ldcs(y + (t * K + k0 + i) * nv + v)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if ((valid >> (k0 + i)) & 1u) {
+                acc.x += a[i].x; acc.y += a[i].y; acc.z += a[i].z; acc.w += a[i].w;
+            }
         }
     }
     uint2 o;
