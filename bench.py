@@ -29,6 +29,7 @@ all ranks.
 on the host cores for the same metric and workload.
 """
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -72,6 +73,29 @@ def layer_alg(idx, T, H, F, K):
 
 
 # ------------------------------------------------------------- rank timing ----
+
+def mapped_host_buffer(nbytes):
+    """(host pointer, device pointer) of a mapped pinned host allocation, or
+    None when the runtime bindings or the mapping are unavailable."""
+    try:
+        import cuda.bindings.runtime as rt
+    except ImportError:
+        return None
+    ok = rt.cudaError_t.cudaSuccess
+    err, hp = rt.cudaHostAlloc(nbytes, rt.cudaHostAllocMapped | rt.cudaHostAllocPortable)
+    if err != ok:
+        return None
+    err, dp = rt.cudaHostGetDevicePointer(hp, 0)
+    if err != ok or not dp:
+        rt.cudaFreeHost(hp)
+        return None
+    return int(hp), int(dp)
+
+
+def free_mapped_host_buffer(hp):
+    import cuda.bindings.runtime as rt
+    rt.cudaFreeHost(hp)
+
 
 def max_over_ranks(v, world, device):
     """Largest value over all ranks (identity on one rank)."""
@@ -235,23 +259,65 @@ def run_ours(args):
     launches_per_step = 2
 
     # ---- end to end through the C ABI with host buffers -------------------
-    xh = lay1.x.cpu().pin_memory()
-    ih = lay1.idx.cpu().pin_memory()
-    wh = lay1.w.cpu().pin_memory()
-    oh = torch.empty_like(out1, device="cpu").pin_memory()
-    xd, idd, wd = torch.empty_like(lay1.x), torch.empty_like(lay1.idx), torch.empty_like(lay1.w)
+    # The step's inputs (x, top-k ids, top-k weights) sit in one pinned host
+    # buffer and go over in one copy; the step (copy in, decode, copy out) is
+    # captured once and replayed, as a serving loop would.
+    def packed(tensors):
+        offs, o = [], 0
+        for t_ in tensors:
+            offs.append(o)
+            o += (t_.numel() * t_.element_size() + 255) // 256 * 256
+        return offs, o
+    ins = [lay1.x, lay1.idx, lay1.w]
+    offs, nbytes = packed(ins)
+    hbuf = torch.zeros(nbytes, dtype=torch.uint8).pin_memory()
+    dbuf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    views_d = []
+    for t_, o in zip(ins, offs):
+        nb = t_.numel() * t_.element_size()
+        hbuf[o:o + nb].copy_(t_.cpu().contiguous().view(-1).view(torch.uint8))
+        views_d.append(dbuf[o:o + nb].view(t_.dtype).view(t_.shape))
+    xd, idd, wd = views_d
+    # The output goes straight into mapped pinned host memory (the kernels
+    # write it over the bus; the C ABI takes any device-accessible pointer).
+    out_bytes = out1.numel() * 2
+    mapped = mapped_host_buffer(out_bytes)
+    if mapped is not None:
+        h_out, d_out = mapped
+        C = ctypes.c_void_p
 
-    def e2e_call():
-        xd.copy_(xh, non_blocking=True)
-        idd.copy_(ih, non_blocking=True)
-        wd.copy_(wh, non_blocking=True)
-        moe.moe_experts_decode(xd, lay1.gate_up, lay1.down, idd, wd, K, out=out1, workspace=ws1)
-        oh.copy_(out1, non_blocking=True)
+        def e2e_call():
+            dbuf.copy_(hbuf, non_blocking=True)
+            rc = moe.lib.moe_experts_decode(
+                C(xd.data_ptr()), C(lay1.gate_up.data_ptr()), C(lay1.down.data_ptr()),
+                C(idd.data_ptr()), C(wd.data_ptr()), K, 1, H, F, E, 0, None, None, C(d_out),
+                C(ws1.data_ptr()), ws1.numel(), C(torch.cuda.current_stream().cuda_stream))
+            assert rc == 0, rc
+        e2e_how = "one copy of the pinned inputs, decode writing out into mapped pinned host memory"
+    else:
+        oh = torch.empty_like(out1, device="cpu").pin_memory()
 
-    e2e_times = time_eager(e2e_call, args.steps, args.warmup)
+        def e2e_call():
+            dbuf.copy_(hbuf, non_blocking=True)
+            moe.moe_experts_decode(xd, lay1.gate_up, lay1.down, idd, wd, K, out=out1, workspace=ws1)
+            oh.copy_(out1, non_blocking=True)
+        e2e_how = "one copy of the pinned inputs, decode, one copy of out to pinned host memory"
+
+    e2e_times, e2e_graph = time_graph(e2e_call, args.steps, args.warmup)
     e2e_us = per_layer_us(rank_max(sum(e2e_times)), args.steps, world)
-    h2d = xh.numel() * 2 + ih.numel() * 4 + wh.numel() * 4
-    d2h = oh.numel() * 2
+    h2d = sum(t_.numel() * t_.element_size() for t_ in ins)
+    d2h = out_bytes
+    if mapped is not None:
+        # the replayed step itself must produce the output: clear, replay, compare
+        torch.cuda.synchronize()
+        ctypes.memset(h_out, 0, out_bytes)
+        e2e_graph.replay()
+        torch.cuda.synchronize()
+        host_out = np.frombuffer(ctypes.string_at(h_out, out_bytes), dtype=np.uint16)
+        dev_out = out1.view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
+        assert np.array_equal(host_out, dev_out), "replayed step did not write the output"
+        free_mapped_host_buffer(h_out)
+    del e2e_graph
 
     # ---- breakdown: other decode sizes, eager decode, OCR-2 prefill ---------
     breakdown = {}
@@ -364,7 +430,9 @@ def run_ours(args):
                      "frac": round(achieved / peaks["hbm"], 4), "traffic": traffic,
                      "algorithmic_bytes": alg1["bytes"], "peak_source": peaks["source"]},
         "e2e": {"value": round(e2e_us, 3), "unit": "us/layer", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "timing": e2e_how + "; the step captured in a CUDA graph and replayed, L2 "
+                          "flushed before each"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "breakdown": breakdown,

@@ -95,7 +95,9 @@ MOE_API size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe
  *   gate_up_scale  [E,2F,H/128] fp32 (e4m3 only; NULL for bf16): the value of
  *                  gate_up element (e,r,c) is e4m3(q) * gate_up_scale[e,r,c/128]
  *   down_scale     [E,H,F/128]  fp32 (e4m3 only; NULL for bf16)
- *   out            [T,H]     bf16, fully overwritten
+ *   out            [T,H]     bf16, fully overwritten (any device-accessible
+ *                            pointer, e.g. mapped pinned host memory: the
+ *                            kernels store it directly)
  *   workspace      device scratch of >= moe_experts_workspace_size(..., 0)
  *                  bytes, 256-byte aligned; contents need no initialisation
  *
