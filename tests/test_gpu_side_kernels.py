@@ -50,7 +50,8 @@ def test_router_bit_exact(moe, cuda_dev, T, E, G, TG, K):
 
 
 @pytest.mark.parametrize("T,K,E,skew", [(1, 6, 64, None), (16, 6, 64, None), (2048, 6, 64, None),
-                                        (777, 8, 256, 1.1), (8192, 8, 256, 1.1), (5, 4, 1024, None)])
+                                        (777, 8, 256, 1.1), (8192, 8, 256, 1.1), (5, 4, 1024, None),
+                                        (512, 8, 64, None), (513, 8, 64, None)])   # 4096 / 4104 slots
 def test_permute_bit_exact(moe, cuda_dev, T, K, E, skew):
     lay = inputs.ocr2_layer(T, seed=T, device="cpu", H=128, F=128, E=E, K=K, zipf=skew)
     idx = lay.idx.clone()
