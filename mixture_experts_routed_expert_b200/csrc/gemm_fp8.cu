@@ -146,7 +146,10 @@ __global__ void __launch_bounds__(kThreads8, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
+            // weight tiles: evict-first when only this tile reads them, kept
+            // (evict-last) when the expert's other routed-row tiles, running
+            // on neighbouring SMs at the same time, read them too
+            const uint64_t pol_once = policy_evict_first();
             const uint64_t pol_x = policy_evict_last();
             int stage = 0, armed[C::MAX_STAGES];
             uint32_t phase = 0;
@@ -154,6 +157,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
             bool ok = true;
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
+                const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
                 const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
                 const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * C::BOX * 128;
                 const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
