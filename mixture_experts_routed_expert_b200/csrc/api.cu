@@ -72,16 +72,14 @@ Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t w
 }
 
 DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t wt) {
+    (void)H;
     (void)E;
+    (void)wt;                        // only bf16 weights take the gather-GEMV kernels
     const size_t N = (size_t)T * K;
     DecodeWorkspace L;
     Bump b;
-    L.sync = b.take(sizeof(int32_t) * decode_sync_ints(H));
+    L.sync = b.take(sizeof(int32_t) * 4);
     L.h = b.take(2 * N * F);
-    L.ys = b.take(0);
-    (void)wt;                        // the E4M3 kernels quantise h in shared memory
-    L.hq = b.take(0);
-    L.hscale = b.take(0);
     L.total = b.off;
     return L;
 }

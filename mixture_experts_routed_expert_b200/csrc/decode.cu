@@ -307,11 +307,6 @@ cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *d
 
 namespace moe {
 
-size_t decode_sync_ints(int H) {
-    (void)H;
-    return 4;
-}
-
 // The decode kernels keep every intermediate in registers and small shared
 // arrays; the only shape limit is the per-lane vector count of one row.
 bool decode_shape_ok(int H, int F) { return H / 8 <= 32 * 8 && F / 8 <= 32 * 8; }

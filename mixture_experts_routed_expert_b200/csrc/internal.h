@@ -37,15 +37,10 @@ struct Workspace {
 Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t wt);
 
 struct DecodeWorkspace {
-    size_t sync;          // int32: status word (+3 spare)
-    size_t h;             // [T*K][F] bf16
-    size_t ys;            // unused (kept empty)
-    size_t hq;            // [T*K][F] e4m3 (e4m3 path)
-    size_t hscale;        // [T*K][F/128] f32 (e4m3 path)
+    size_t sync;          // int32 status words (4)
+    size_t h;             // [T*K][F] bf16, by slot
     size_t total;
 };
-// int32 entries of the decode sync region for hidden size H.
-size_t decode_sync_ints(int H);
 // True when the decode kernel's shared-memory staging fits these sizes.
 bool decode_shape_ok(int H, int F);
 DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t wt);
