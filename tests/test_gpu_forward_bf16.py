@@ -109,3 +109,23 @@ def test_prefill_ocr2_zipf_sweep_sampled(moe, cuda_dev, ocr_weights, T):
     rows = torch.nonzero((lay.idx == hot).any(dim=1)).reshape(-1)
     tokens = torch.unique(torch.cat([rows[:8], torch.tensor([0, T - 1])]))
     assert_matches_oracle(out[tokens.to(out.device)], _ref(lay, tokens), "prefill zipf T=%d" % T)
+
+
+@pytest.mark.parametrize("T", [1, 5, 16, 17])
+def test_prefill_few_tokens_invalid_slots(moe, cuda_dev, ocr_weights, T):
+    """Few tokens through the grouped GEMMs: a token whose slots are all
+    invalid, repeated calls, and a call where no slot is valid (no tiles)."""
+    lay = inputs.ocr2_layer(T, seed=90 + T, device="cpu", weights_from=ocr_weights)
+    if T > 1:
+        lay.idx[1, :] = -1
+    out = _run(moe, lay, cuda_dev, "moe_experts_prefill")
+    assert_matches_oracle(out, _ref(lay), "prefill T=%d invalid slots" % T)
+    if T > 1:
+        assert torch.count_nonzero(out[1].float()) == 0
+    for _ in range(2):                       # deterministic across calls
+        assert torch.equal(_run(moe, lay, cuda_dev, "moe_experts_prefill"), out)
+    lay.idx.fill_(-1)
+    out0 = torch.full((T, 1280), float("nan"), dtype=torch.bfloat16, device=cuda_dev)
+    out0 = moe.moe_experts_prefill(lay.x.to(cuda_dev), lay.gate_up.to(cuda_dev), lay.down.to(cuda_dev),
+                                   lay.idx.to(cuda_dev), lay.w.to(cuda_dev), 6, out=out0)
+    assert torch.count_nonzero(out0.float()) == 0

@@ -140,3 +140,19 @@ def test_fp8_dsv3_decode_sampled(moe, cuda_dev, dsv3_weights, T):
     tokens = torch.arange(T) if T <= 4 else torch.tensor([0, 3, T - 1])
     assert_matches_oracle(out[tokens.to(out.device)], _oracle(lay, idx, w, tokens),
                           "fp8 DSV3 decode T=%d" % T)
+
+
+@pytest.mark.parametrize("T", [3, 16])
+def test_fp8_few_tokens_invalid_slots(moe, cuda_dev, T):
+    """Few tokens on E4M3 weights through both entries, with an all-invalid
+    token and an all-invalid call."""
+    lay = inputs.fp8_layer(T, seed=300 + T, device="cpu", H=512, F=256, E=16)
+    idx, w = _route(lay, 4)
+    idx[1, :] = -1
+    for fn in ("moe_experts_prefill", "moe_experts_decode"):
+        out = _run(moe, lay, idx, w, cuda_dev, fn)
+        assert_matches_oracle(out, _oracle(lay, idx, w), "fp8 T=%d %s" % (T, fn))
+        assert torch.count_nonzero(out[1].float()) == 0
+    idx.fill_(-1)
+    out = _run(moe, lay, idx, w, cuda_dev)
+    assert torch.count_nonzero(out.float()) == 0
