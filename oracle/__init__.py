@@ -40,6 +40,10 @@ def lib():
         L.oracle_permute.argtypes = [P, i64, i32, P, P, P, P]
         L.oracle_moe_forward_bf16.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i32, P]
         L.oracle_moe_forward_fp8.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, P]
+        L.oracle_moe_forward_shared_bf16.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i32, P, P,
+                                                     i32, P, P]
+        L.oracle_moe_forward_shared_fp8.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, P,
+                                                    P, P, P, i32, P, P]
         L.oracle_num_threads.restype = ctypes.c_int
         for fn in ("oracle_bf16_from_f64", "oracle_e4m3_from_f64", "oracle_e4m3_to_f64",
                    "oracle_quantize_fp8_block128", "oracle_route_sigmoid_grouped",
@@ -167,4 +171,56 @@ def moe_forward_fp8(x, w13, w13_scale, w2, w2_scale, idx, w):
     out = np.empty((T, H), np.uint16)
     lib().oracle_moe_forward_fp8(px, pa, psa, pb, psb, pi, pw, T, H, F, E, ix.shape[1],
                                  out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def moe_forward_shared_bf16(x, gate_up, down, idx, w, shared_gate_up, shared_down, residual=None):
+    """Routed + shared experts + residual, bf16 weights: shared_gate_up
+    [S,2F,H], shared_down [S,H,F], residual [T,H] (bf16 bits) or None."""
+    x, px = _c(x, np.uint16)
+    gu, pg = _c(gate_up, np.uint16)
+    dn, pd = _c(down, np.uint16)
+    ix, pi = _c(idx, np.int32)
+    ww, pw = _c(w, np.float32)
+    sg, psg = _c(shared_gate_up, np.uint16)
+    sd, psd = _c(shared_down, np.uint16)
+    T, H = x.shape
+    E, F2, _ = gu.shape
+    S = sg.shape[0]
+    assert sg.shape[1:] == (F2, H) and sd.shape == (S, H, F2 // 2)
+    pr = None
+    if residual is not None:
+        r, pr = _c(residual, np.uint16)
+        assert r.shape == (T, H)
+    out = np.empty((T, H), np.uint16)
+    lib().oracle_moe_forward_shared_bf16(px, pg, pd, pi, pw, T, H, F2 // 2, E, ix.shape[1], psg, psd,
+                                         S, pr, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def moe_forward_shared_fp8(x, w13, w13_scale, w2, w2_scale, idx, w, sw13, sw13_scale, sw2,
+                           sw2_scale, residual=None):
+    """Routed + shared experts + residual, E4M3 weights with per-(row,128) scales."""
+    x, px = _c(x, np.uint16)
+    a, pa = _c(w13, np.uint8)
+    sa, psa = _c(w13_scale, np.float32)
+    b, pb = _c(w2, np.uint8)
+    sb, psb = _c(w2_scale, np.float32)
+    ix, pi = _c(idx, np.int32)
+    ww, pw = _c(w, np.float32)
+    c, pc = _c(sw13, np.uint8)
+    sc, psc = _c(sw13_scale, np.float32)
+    d, pdd = _c(sw2, np.uint8)
+    sd, psd = _c(sw2_scale, np.float32)
+    T, H = x.shape
+    E, F2, _ = a.shape
+    S = c.shape[0]
+    assert c.shape[1:] == (F2, H) and d.shape == (S, H, F2 // 2)
+    pr = None
+    if residual is not None:
+        r, pr = _c(residual, np.uint16)
+        assert r.shape == (T, H)
+    out = np.empty((T, H), np.uint16)
+    lib().oracle_moe_forward_shared_fp8(px, pa, psa, pb, psb, pi, pw, T, H, F2 // 2, E, ix.shape[1],
+                                        pc, psc, pdd, psd, S, pr, out.ctypes.data_as(ctypes.c_void_p))
     return out

@@ -145,3 +145,36 @@ def forward_fp8(x, w13, w13_scale, w2, w2_scale, idx, w):
                 terms[j].append(w[t][k] * y)
         out.append([bf16_round(math.fsum(terms[j])) for j in range(H)])
     return out
+
+
+def forward_shared_bf16(x, gate_up, down, idx, w, shared_gate_up, shared_down, residual):
+    """Routed + shared experts (weight 1, every token) + residual, bf16
+    weights; one exact sum per output (math.fsum), rounded to bf16 once."""
+    T, H = len(x), len(x[0])
+    E = len(gate_up)
+    F = len(gate_up[0]) // 2
+
+    def expert_terms(G, D, t, wk):
+        hvec = []
+        for f in range(F):
+            g = math.fsum(G[f][i] * x[t][i] for i in range(H))
+            u = math.fsum(G[F + f][i] * x[t][i] for i in range(H))
+            hvec.append(bf16_round(silu(g) * u))
+        return [wk * math.fsum(D[j][f] * hvec[f] for f in range(F)) for j in range(H)]
+
+    out = []
+    for t in range(T):
+        terms = [[] for _ in range(H)]
+        for k in range(len(idx[t])):
+            e = idx[t][k]
+            if 0 <= e < E:
+                for j, v in enumerate(expert_terms(gate_up[e], down[e], t, w[t][k])):
+                    terms[j].append(v)
+        for s in range(len(shared_gate_up)):
+            for j, v in enumerate(expert_terms(shared_gate_up[s], shared_down[s], t, 1.0)):
+                terms[j].append(v)
+        if residual is not None:
+            for j in range(H):
+                terms[j].append(residual[t][j])
+        out.append([bf16_round(math.fsum(terms[j])) for j in range(H)])
+    return out

@@ -258,13 +258,41 @@ void oracle_permute(const int32_t *idx, int64_t n_slots, int E, int32_t *counts,
 
 static double silu(double g) { return g / (1.0 + exp(-g)); }
 
-/* bf16 weights.  x [T,H], gate_up [E,2F,H] (rows [0,F) gate, [F,2F) up),
- * down [E,H,F], idx/w [T,K]; out [T,H] bf16.
- * h is rounded to bf16 (the intermediate activation is stored in the
- * activation dtype); y is not rounded; out = bf16(sum_k w y). */
-void oracle_moe_forward_bf16(const uint16_t *x, const uint16_t *gate_up, const uint16_t *down,
-                             const int32_t *idx, const float *w, int64_t T, int H, int F, int E,
-                             int K, uint16_t *out) {
+/* One expert's contribution for one token, bf16 weights: gate rows G [F,H],
+ * up rows U [F,H], down D [H,F]; xt = x_t (exact bf16 values).
+ * h_f = bf16(SiLU(g_f) u_f); acc_j += wk * sum_f D[j,f] h_f (fp64, ascending
+ * indices).  hb: scratch [F]. */
+static void contrib_bf16(const double *xt, const uint16_t *G, const uint16_t *U, const uint16_t *D,
+                         int H, int F, double wk, double *hb, double *acc) {
+    for (int f = 0; f < F; ++f) {
+        double g = 0.0, u = 0.0;
+        for (int i = 0; i < H; ++i) {
+            g += bf16_value(G[(int64_t)f * H + i]) * xt[i];
+            u += bf16_value(U[(int64_t)f * H + i]) * xt[i];
+        }
+        hb[f] = bf16_value(bf16_from_double(silu(g) * u));
+    }
+    for (int j = 0; j < H; ++j) {
+        double y = 0.0;
+        for (int f = 0; f < F; ++f) y += bf16_value(D[(int64_t)j * F + f]) * hb[f];
+        acc[j] += wk * y;
+    }
+}
+
+/* Routed experts plus S shared experts and a residual, bf16 weights.
+ *   out[t] = bf16( sum_k w[t,k] E_{idx[t,k]}(x_t) + sum_s Shared_s(x_t) + residual[t] )
+ * summed in fp64 in that order (k ascending, then s ascending, then the
+ * residual), rounded once.  Each shared expert is a SwiGLU MLP of width F
+ * applied to every token with weight 1 ("Supporting MegaKernel for DeepSeek
+ * Models": shared expert through silu_mul_layer; moe_local_reduction adds the
+ * residual to the weighted sum).  shared_gate_up [S,2F,H], shared_down
+ * [S,H,F]; residual [T,H] bf16 or NULL; S = 0 and NULL give the routed
+ * forward alone. */
+void oracle_moe_forward_shared_bf16(const uint16_t *x, const uint16_t *gate_up, const uint16_t *down,
+                                    const int32_t *idx, const float *w, int64_t T, int H, int F,
+                                    int E, int K, const uint16_t *shared_gate_up,
+                                    const uint16_t *shared_down, int S, const uint16_t *residual,
+                                    uint16_t *out) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t t = 0; t < T; ++t) {
         double *xt = (double *)malloc(sizeof(double) * H);
@@ -275,37 +303,68 @@ void oracle_moe_forward_bf16(const uint16_t *x, const uint16_t *gate_up, const u
             int e = idx[t * K + k];
             if (e < 0 || e >= E) continue;
             const uint16_t *G = gate_up + (int64_t)e * 2 * F * H;
-            const uint16_t *U = G + (int64_t)F * H;
-            const uint16_t *D = down + (int64_t)e * H * F;
-            for (int f = 0; f < F; ++f) {
-                double g = 0.0, u = 0.0;
-                for (int i = 0; i < H; ++i) {
-                    g += bf16_value(G[(int64_t)f * H + i]) * xt[i];
-                    u += bf16_value(U[(int64_t)f * H + i]) * xt[i];
-                }
-                hb[f] = bf16_value(bf16_from_double(silu(g) * u));
-            }
-            double wk = (double)w[t * K + k];
-            for (int j = 0; j < H; ++j) {
-                double y = 0.0;
-                for (int f = 0; f < F; ++f) y += bf16_value(D[(int64_t)j * F + f]) * hb[f];
-                acc[j] += wk * y;
-            }
+            contrib_bf16(xt, G, G + (int64_t)F * H, down + (int64_t)e * H * F, H, F,
+                         (double)w[t * K + k], hb, acc);
         }
+        for (int s = 0; s < S; ++s) {
+            const uint16_t *G = shared_gate_up + (int64_t)s * 2 * F * H;
+            contrib_bf16(xt, G, G + (int64_t)F * H, shared_down + (int64_t)s * H * F, H, F, 1.0, hb,
+                         acc);
+        }
+        if (residual)
+            for (int j = 0; j < H; ++j) acc[j] += bf16_value(residual[t * H + j]);
         for (int j = 0; j < H; ++j) out[t * H + j] = bf16_from_double(acc[j]);
         free(xt); free(acc); free(hb);
     }
 }
 
-/* FP8 E4M3 weights with fp32 scales per (row, 128-column block):
- * w13 [E,2F,H] + w13_scale [E,2F,H/128], w2 [E,H,F] + w2_scale [E,H,F/128].
- * x (bf16) is quantised per 128 columns by the S2 rule; h = bf16(SiLU(g) u)
- * is quantised per 128 features by the same rule; every E4M3 operand is
- * dequantised (code value * its block scale) before the fp64 dot products;
- * out = bf16(sum_k w y). */
-void oracle_moe_forward_fp8(const uint16_t *x, const uint8_t *w13, const float *w13_scale,
-                            const uint8_t *w2, const float *w2_scale, const int32_t *idx,
-                            const float *w, int64_t T, int H, int F, int E, int K, uint16_t *out) {
+/* bf16 weights.  x [T,H], gate_up [E,2F,H] (rows [0,F) gate, [F,2F) up),
+ * down [E,H,F], idx/w [T,K]; out [T,H] bf16.
+ * h is rounded to bf16 (the intermediate activation is stored in the
+ * activation dtype); y is not rounded; out = bf16(sum_k w y). */
+void oracle_moe_forward_bf16(const uint16_t *x, const uint16_t *gate_up, const uint16_t *down,
+                             const int32_t *idx, const float *w, int64_t T, int H, int F, int E,
+                             int K, uint16_t *out) {
+    oracle_moe_forward_shared_bf16(x, gate_up, down, idx, w, T, H, F, E, K, NULL, NULL, 0, NULL, out);
+}
+
+/* One expert's contribution for one token, E4M3 weights with fp32 scales per
+ * (row, 128 columns): W13 [2F,H] + S13 [2F,H/128], W2 [H,F] + S2 [H,F/128];
+ * xd = the token's quantised-dequantised activations.  h = bf16(SiLU(g) u)
+ * is quantised per 128 features by the S2 rule and dequantised before the
+ * down projection.  Scratch: hv, hd [F], hq [F], hs [F/128]. */
+static void contrib_fp8(const double *xd, const double *lut, const uint8_t *W13, const float *S13,
+                        const uint8_t *W2, const float *S2, int H, int F, double wk, double *hv,
+                        double *hd, uint8_t *hq, float *hs, double *acc) {
+    int hb_n = H / 128, fb_n = F / 128;
+    for (int f = 0; f < F; ++f) {
+        int64_t rg = f, ru = (int64_t)F + f;
+        double g = 0.0, u = 0.0;
+        for (int i = 0; i < H; ++i) {
+            g += lut[W13[rg * H + i]] * (double)S13[rg * hb_n + i / 128] * xd[i];
+            u += lut[W13[ru * H + i]] * (double)S13[ru * hb_n + i / 128] * xd[i];
+        }
+        hv[f] = bf16_value(bf16_from_double(silu(g) * u));
+    }
+    quantize_blocks(hv, fb_n, hq, hs);
+    for (int f = 0; f < F; ++f) hd[f] = e4m3_value(hq[f]) * (double)hs[f / 128];
+    for (int j = 0; j < H; ++j) {
+        double y = 0.0;
+        for (int f = 0; f < F; ++f)
+            y += lut[W2[(int64_t)j * F + f]] * (double)S2[(int64_t)j * fb_n + f / 128] * hd[f];
+        acc[j] += wk * y;
+    }
+}
+
+/* Routed experts plus S shared experts and a residual, E4M3 weights (same
+ * order and rounding points as oracle_moe_forward_shared_bf16; every E4M3
+ * operand dequantised before the fp64 dot products). */
+void oracle_moe_forward_shared_fp8(const uint16_t *x, const uint8_t *w13, const float *w13_scale,
+                                   const uint8_t *w2, const float *w2_scale, const int32_t *idx,
+                                   const float *w, int64_t T, int H, int F, int E, int K,
+                                   const uint8_t *sw13, const float *sw13_scale, const uint8_t *sw2,
+                                   const float *sw2_scale, int S, const uint16_t *residual,
+                                   uint16_t *out) {
     int hb_n = H / 128, fb_n = F / 128;
     double lut[256];                               /* value of every E4M3 code */
     for (int c = 0; c < 256; ++c) lut[c] = e4m3_value((uint8_t)c);
@@ -326,29 +385,32 @@ void oracle_moe_forward_fp8(const uint16_t *x, const uint8_t *w13, const float *
         for (int k = 0; k < K; ++k) {
             int e = idx[t * K + k];
             if (e < 0 || e >= E) continue;
-            for (int f = 0; f < F; ++f) {
-                int64_t rg = (int64_t)e * 2 * F + f, ru = rg + F;
-                double g = 0.0, u = 0.0;
-                for (int i = 0; i < H; ++i) {
-                    g += lut[w13[rg * H + i]] * (double)w13_scale[rg * hb_n + i / 128] * xd[i];
-                    u += lut[w13[ru * H + i]] * (double)w13_scale[ru * hb_n + i / 128] * xd[i];
-                }
-                hv[f] = bf16_value(bf16_from_double(silu(g) * u));
-            }
-            quantize_blocks(hv, fb_n, hq, hs);
-            for (int f = 0; f < F; ++f) hd[f] = e4m3_value(hq[f]) * (double)hs[f / 128];
-            double wk = (double)w[t * K + k];
-            for (int j = 0; j < H; ++j) {
-                int64_t rd = (int64_t)e * H + j;
-                double y = 0.0;
-                for (int f = 0; f < F; ++f)
-                    y += lut[w2[rd * F + f]] * (double)w2_scale[rd * fb_n + f / 128] * hd[f];
-                acc[j] += wk * y;
-            }
+            contrib_fp8(xd, lut, w13 + (int64_t)e * 2 * F * H, w13_scale + (int64_t)e * 2 * F * hb_n,
+                        w2 + (int64_t)e * H * F, w2_scale + (int64_t)e * H * fb_n, H, F,
+                        (double)w[t * K + k], hv, hd, hq, hs, acc);
         }
+        for (int s = 0; s < S; ++s)
+            contrib_fp8(xd, lut, sw13 + (int64_t)s * 2 * F * H, sw13_scale + (int64_t)s * 2 * F * hb_n,
+                        sw2 + (int64_t)s * H * F, sw2_scale + (int64_t)s * H * fb_n, H, F, 1.0, hv, hd,
+                        hq, hs, acc);
+        if (residual)
+            for (int j = 0; j < H; ++j) acc[j] += bf16_value(residual[t * H + j]);
         for (int j = 0; j < H; ++j) out[t * H + j] = bf16_from_double(acc[j]);
         free(xt); free(xd); free(xq); free(xs); free(acc); free(hv); free(hd); free(hq); free(hs);
     }
+}
+
+/* FP8 E4M3 weights with fp32 scales per (row, 128-column block):
+ * w13 [E,2F,H] + w13_scale [E,2F,H/128], w2 [E,H,F] + w2_scale [E,H,F/128].
+ * x (bf16) is quantised per 128 columns by the S2 rule; h = bf16(SiLU(g) u)
+ * is quantised per 128 features by the same rule; every E4M3 operand is
+ * dequantised (code value * its block scale) before the fp64 dot products;
+ * out = bf16(sum_k w y). */
+void oracle_moe_forward_fp8(const uint16_t *x, const uint8_t *w13, const float *w13_scale,
+                            const uint8_t *w2, const float *w2_scale, const int32_t *idx,
+                            const float *w, int64_t T, int H, int F, int E, int K, uint16_t *out) {
+    oracle_moe_forward_shared_fp8(x, w13, w13_scale, w2, w2_scale, idx, w, T, H, F, E, K, NULL, NULL,
+                                  NULL, NULL, 0, NULL, out);
 }
 
 #ifdef _OPENMP
