@@ -400,12 +400,37 @@ def run_ours(args):
         tc_frac=round(t_tc / us, 3), hbm_frac=round(t_hbm / us, 3),
         roofline_frac=round(max(t_hbm, t_tc) / us, 3), bound="hbm" if t_hbm > t_tc else "tensor")
     del g
+    # OCR-2 layer with its 2 shared experts and a residual (one call)
+    sgu, sdn = inputs.shared_experts_bf16(2, H, F, seed=1, device=dev)
+    for T in (1, 2048):
+        lay = inputs.ocr2_layer(T, seed=T, device=dev, weights_from=base)
+        res = inputs.residual_bf16(T, H, seed=T, device=dev)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(moe.moe_experts_shared_workspace_size(T, H, F, E, K, 2, 0),
+                         dtype=torch.uint8, device=dev)
+        call = lambda: moe.moe_experts_with_shared(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K,
+                                                   sgu, sdn, residual=res, out=out, workspace=ws)
+        t, g = time_graph(call, args.steps, args.warmup)
+        us = float(np.mean(t))
+        a = layer_alg(lay.idx.cpu().numpy(), T, H, F, K)
+        n_t = a["touched_experts"] + 2
+        byts = n_t * 3 * H * F * 2 + T * H * 6
+        flops = 6 * T * (K + 2) * H * F
+        t_hbm = byts / (peaks["hbm"] * 1e3)
+        t_tc = flops / (peaks["bf16"] * 1e6)
+        breakdown["bf16_shared2_residual_T%d" % T] = dict(
+            us=round(us, 2), touched_experts=n_t, gbs=round(byts / us / 1e3, 1),
+            tflops=round(flops / us / 1e6, 1), roofline_frac=round(max(t_hbm, t_tc) / us, 3),
+            bound="hbm" if t_hbm > t_tc else "tensor", entry="with_shared")
+        del g
+    del sgu, sdn
     # ---- DeepSeek-V3-like FP8 layer: group-sigmoid router + E4M3 experts ----
     fp8_w = inputs.fp8_weights(seed=0, device=dev)
     D = inputs.DSV3_FP8
     per_expert_fp8 = (3 * D["F"] * D["H"]) + 4 * (3 * D["F"] * D["H"] // 128)
 
-    def fp8_entry(T, zipf, steps):
+    def fp8_entry(T, zipf, steps, S=0):
+        """S > 0: moe_experts_with_shared with S shared experts and a residual."""
         lay = inputs.fp8_layer(T, seed=T, device=dev, weights=fp8_w, zipf=zipf)
         idx = torch.empty(T, D["K"], dtype=torch.int32, device=dev)
         tw = torch.empty(T, D["K"], dtype=torch.float32, device=dev)
@@ -414,6 +439,18 @@ def run_ours(args):
         wsz = moe.moe_experts_workspace_size(T, D["H"], D["F"], D["E"], D["K"], 1, dec)
         ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
         fn = moe.moe_experts_decode if dec else moe.moe_experts_prefill
+        if S > 0:
+            sh = inputs.shared_experts_fp8(S, D["H"], D["F"], seed=1, device=dev)
+            res = inputs.residual_bf16(T, D["H"], seed=T, device=dev)
+            ws = torch.empty(moe.moe_experts_shared_workspace_size(T, D["H"], D["F"], D["E"], D["K"],
+                                                                   S, 1),
+                             dtype=torch.uint8, device=dev)
+
+            def fn(x, w13, w2, i, w, K, gate_up_scale, down_scale, out, workspace):
+                moe.moe_experts_with_shared(x, w13, w2, i, w, K, sh[0], sh[2], residual=res,
+                                            gate_up_scale=gate_up_scale, down_scale=down_scale,
+                                            shared_gate_up_scale=sh[1], shared_down_scale=sh[3],
+                                            out=out, workspace=workspace)
 
         def call():
             moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"], D["topk_group"],
@@ -422,9 +459,9 @@ def run_ours(args):
                down_scale=lay.w2_scale, out=out, workspace=ws)
         t, g = time_graph(call, steps, args.warmup)
         us = float(np.mean(t))
-        n_t = len(set(idx.cpu().reshape(-1).tolist()))
-        byts = n_t * per_expert_fp8 + T * D["H"] * 4 + T * D["E"] * 4
-        flops = 6 * T * D["K"] * D["H"] * D["F"]
+        n_t = len(set(idx.cpu().reshape(-1).tolist())) + S
+        byts = n_t * per_expert_fp8 + T * D["H"] * (4 + 2 * (S > 0)) + T * D["E"] * 4
+        flops = 6 * T * (D["K"] + S) * D["H"] * D["F"]
         t_hbm = byts / (peaks["hbm"] * 1e3)
         t_tc = flops / (2 * peaks["bf16"] * 1e6)
         del g
@@ -437,6 +474,11 @@ def run_ours(args):
         breakdown["fp8_dsv3_T%d" % T] = dict(fp8_entry(T, None, args.steps),
                                              entry="decode" if T * D["K"] <= 64 else "prefill",
                                              includes="router + quantise + experts")
+    # one shared expert and a residual folded into the same grouped GEMMs
+    for T in (128, 8):
+        breakdown["fp8_dsv3_shared1_residual_T%d" % T] = dict(
+            fp8_entry(T, None, args.steps, S=1), entry="with_shared",
+            includes="router + quantise + routed and shared experts + residual")
     # skewed sweep (Zipf 1.1 expert popularity), FP8 and the OCR-2 bf16 shape
     sweep_steps = max(3, min(args.steps, 10))
     sweep = {}

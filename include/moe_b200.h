@@ -133,6 +133,51 @@ MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *g
                                 size_t workspace_bytes, void *stream);
 
 /*
+ * Bytes of workspace needed by moe_experts_with_shared for these sizes
+ * (0 when the sizes are invalid).
+ */
+MOE_API size_t moe_experts_shared_workspace_size(int T, int H, int F, int E, int K, int S,
+                                                 moe_wtype_t wt);
+
+/*
+ * Routed experts, S shared experts and a residual in one call: the expert
+ * layer of a DeepSeek-style model with the two steps either side of the
+ * routed op folded in ("Supporting MegaKernel for DeepSeek Models": the shared
+ * expert is a SwiGLU MLP applied to every token; moe_local_reduction adds a
+ * residual to the weighted sum of the expert rows):
+ *
+ *   out[t] = bf16( sum_{k<K} w[t,k] E_{idx[t,k]}(x_t)
+ *                  + sum_{s<S} Shared_s(x_t) + residual[t] )
+ *
+ * summed in fp32 in that order (k ascending, then s, then the residual) and
+ * rounded once.  Each shared expert has the routed experts' width F and the
+ * same projections; a shared MLP of width S*F is the sum of S such experts
+ * (split its rows into S blocks of F).  The shared experts run as S extra
+ * expert ids of the same grouped GEMMs (every token gets them with weight
+ * 1), so their rows share the routed experts' tiles, pipeline and
+ * precision (e4m3: the same activation quantisation and block scales).
+ *
+ *   arguments shared with moe_experts_prefill: same meaning and layouts
+ *   shared_gate_up_proj  [S,2F,H] bf16 | e4m3 (same dtype as the routed weights)
+ *   shared_down_proj     [S,H,F]  bf16 | e4m3
+ *   shared_gate_up_scale [S,2F,H/128] fp32 (e4m3 only; NULL for bf16)
+ *   shared_down_scale    [S,H,F/128]  fp32 (e4m3 only; NULL for bf16)
+ *   S                    0 <= S, K + S <= 16, E + S <= 1024
+ *                        (S = 0: routed experts plus the residual)
+ *   residual             [T,H] bf16 or NULL (no residual)
+ *   workspace            >= moe_experts_shared_workspace_size(T,H,F,E,K,S,wt)
+ *                        bytes, 256-byte aligned
+ * All pointers must be 16-byte aligned.
+ */
+MOE_API moe_status_t moe_experts_with_shared(
+    const void *hidden_states, const void *gate_up_proj, const void *down_proj,
+    const int32_t *top_k_index, const float *top_k_weights, int top_k, int T, int H, int F, int E,
+    moe_wtype_t wt, const float *gate_up_scale, const float *down_scale,
+    const void *shared_gate_up_proj, const void *shared_down_proj,
+    const float *shared_gate_up_scale, const float *shared_down_scale, int S,
+    const void *residual, void *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Decode form without a workspace, for callers that cannot allocate device
  * memory where they run the layer: code recorded into a CUDA graph while
  * capture forbids allocation, serving loops and real-time hosts that fix

@@ -6,7 +6,7 @@ pointers, the current CUDA stream -- and calls the C entry point of the same
 name; all arithmetic runs in the library's CUDA kernels.  torch is used for
 device memory (outputs, workspaces) and streams only.
 
-The library must be built (``python -m mixture_experts_routed_expert_b200.build``
+The library must be built (``python mixture_experts_routed_expert_b200/build.py``
 or ``__graft_entry__.build()``); importing this package without it raises.
 """
 import ctypes
@@ -24,7 +24,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 
 EXPORTS = ("moe_abi_version", "moe_status_string", "moe_experts_workspace_size",
            "moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
-           "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static")
+           "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
+           "moe_experts_shared_workspace_size", "moe_experts_with_shared")
 
 
 def _load():
@@ -44,8 +45,13 @@ def _load():
     L.moe_route_sigmoid_grouped.argtypes = [P, P, I, I, I, I, I, F, P, P, P, P]
     L.quantize_fp8_block128.argtypes = [P, I, I, P, P, P]
     L.moe_debug_permute.argtypes = [P, I, I, I, P, P, P, P, P, Z, P]
+    L.moe_experts_shared_workspace_size.restype = Z
+    L.moe_experts_shared_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    L.moe_experts_with_shared.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P,
+                                          P, P, P, P, I, P, P, P, Z, P]
     for n in ("moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
-              "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static"):
+              "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
+              "moe_experts_with_shared"):
         getattr(L, n).restype = I
     return L
 
@@ -128,6 +134,51 @@ def moe_experts_decode(hidden_states, gate_up_proj, down_proj, top_k_index, top_
     """Routed-experts forward, fused gather-GEMV form for a few tokens."""
     return _forward("moe_experts_decode", hidden_states, gate_up_proj, down_proj, top_k_index,
                     top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream)
+
+
+def moe_experts_shared_workspace_size(T, H, F, E, K, S, wtype=MOE_W_BF16):
+    return int(lib.moe_experts_shared_workspace_size(T, H, F, E, K, S, wtype))
+
+
+def moe_experts_with_shared(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
+                            top_k, shared_gate_up_proj, shared_down_proj, residual=None,
+                            gate_up_scale=None, down_scale=None, shared_gate_up_scale=None,
+                            shared_down_scale=None, out=None, workspace=None, stream=None):
+    """Routed experts + S shared experts (weight 1) + optional residual, summed
+    in that order and rounded once.  shared_* [S,2F,H] / [S,H,F] (S may be 0
+    when both are None).  Returns out [T,H] bf16."""
+    T, H = hidden_states.shape
+    E, F2, _ = gate_up_proj.shape
+    F = F2 // 2
+    if shared_gate_up_proj is None:
+        S = 0
+    else:
+        S = shared_gate_up_proj.shape[0]
+        if tuple(shared_gate_up_proj.shape) != (S, F2, H) or \
+                tuple(shared_down_proj.shape) != (S, H, F) or \
+                shared_gate_up_proj.dtype != gate_up_proj.dtype:
+            raise ValueError("shared experts must be [S,2F,H] / [S,H,F] of the routed dtype")
+    if residual is not None and tuple(residual.shape) != (T, H):
+        raise ValueError("residual must be [T,H]")
+    for t in (hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, gate_up_scale,
+              down_scale, shared_gate_up_proj, shared_down_proj, shared_gate_up_scale,
+              shared_down_scale, residual):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+    wt = _wtype(gate_up_proj)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
+    need = moe_experts_shared_workspace_size(T, H, F, E, top_k, S, wt)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=hidden_states.device)
+    rc = lib.moe_experts_with_shared(
+        _ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj), _ptr(top_k_index),
+        _ptr(top_k_weights), top_k, T, H, F, E, wt, _ptr(gate_up_scale), _ptr(down_scale),
+        _ptr(shared_gate_up_proj), _ptr(shared_down_proj), _ptr(shared_gate_up_scale),
+        _ptr(shared_down_scale), S, _ptr(residual), _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "moe_experts_with_shared")
+    return out
 
 
 def moe_experts_decode_static(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,

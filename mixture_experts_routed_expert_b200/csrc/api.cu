@@ -125,7 +125,8 @@ moe_status_t check_common(const void *x, const void *gu, const void *dn, const i
 moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const int32_t *idx,
                          const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
                          const float *gus, const float *dns, void *out, void *ws, size_t ws_bytes,
-                         cudaStream_t st, int bn8 = kBNFp8) {
+                         cudaStream_t st, int bn8 = kBNFp8, const SharedSet &sh = SharedSet(),
+                         const void *residual = nullptr) {
     const Workspace L = prefill_workspace(T, H, F, E, K, wt);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
@@ -134,10 +135,38 @@ moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const in
     cudaError_t e = fp8 ? launch_permute_gather(x, idx, N, K, H, E, bn8, bn8, wt, wsb, L, st)
                         : launch_permute_gather(x, idx, N, K, H, E, kBNGateUp, kBNDown, wt, wsb, L, st);
     if (e == cudaSuccess)
-        e = fp8 ? launch_gemms_fp8(gu, gus, dn, dns, w, T, H, F, E, K, bn8, wsb, L, st)
-                : launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st);
-    if (e == cudaSuccess) e = launch_combine(idx, T, H, E, K, wsb, L, out, st);
+        e = fp8 ? launch_gemms_fp8(gu, gus, dn, dns, w, T, H, F, E, K, bn8, wsb, L, st, sh)
+                : launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st, sh);
+    if (e == cudaSuccess) e = launch_combine(idx, T, H, E, K, wsb, L, out, st, residual);
     return from_cuda(e);
+}
+
+// Workspace of moe_experts_with_shared: the prefill workspace of E+S experts
+// and K+S slots per token, then the widened routing [T][K+S] (ids, weights).
+// Calls served by the gather-GEMV decode kernels (which widen the routing
+// themselves) use the decode workspace of K+S slots, which is smaller.
+struct SharedLayout {
+    Workspace L;
+    size_t idx2, w2, total;
+};
+SharedLayout shared_workspace(int64_t T, int H, int F, int E, int K, int S, moe_wtype_t wt) {
+    SharedLayout s;
+    s.L = prefill_workspace(T, H, F, E + S, K + S, wt);
+    Bump b;
+    b.off = align_up(s.L.total, 256);
+    const size_t n = (size_t)std::max<int64_t>(T * (K + S), 1);
+    s.idx2 = b.take(sizeof(int32_t) * n);
+    s.w2 = b.take(sizeof(float) * n);
+    s.total = b.off;
+    return s;
+}
+// True when the gather-GEMV decode kernels serve a call with S shared experts.
+bool shared_decode_serves(int64_t T, int H, int F, int K, int S, moe_wtype_t wt) {
+    return T <= kDecodeMaxT && decode_serves((int)T, K + S, H, F, wt);
+}
+bool shared_dims_ok(int64_t T, int H, int F, int E, int K, int S) {
+    return S >= 0 && K + S <= 16 && E + S <= 1024 && dims_ok(T, H, F, E + S, K + S) &&
+           dims_ok(T, H, F, E, K);
 }
 
 }  // namespace
@@ -212,6 +241,64 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
     return from_cuda(launch_decode_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
                                         top_k_weights, T, H, F, E, top_k,
                                         static_cast<uint8_t *>(workspace), L, out, st));
+}
+
+size_t moe_experts_shared_workspace_size(int T, int H, int F, int E, int K, int S,
+                                         moe_wtype_t wt) {
+    if (!shared_dims_ok(T, H, F, E, K, S)) return 0;
+    return shared_workspace(T, H, F, E, K, S, wt).total;
+}
+
+moe_status_t moe_experts_with_shared(
+    const void *hidden_states, const void *gate_up_proj, const void *down_proj,
+    const int32_t *top_k_index, const float *top_k_weights, int top_k, int T, int H, int F, int E,
+    moe_wtype_t wt, const float *gate_up_scale, const float *down_scale,
+    const void *shared_gate_up_proj, const void *shared_down_proj,
+    const float *shared_gate_up_scale, const float *shared_down_scale, int S,
+    const void *residual, void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!shared_dims_ok(T, H, F, E, top_k, S)) return MOE_ERR_INVALID_ARG;
+    moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                  top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
+                                  out);
+    if (s != MOE_OK || T == 0) return s;
+    if (S > 0) {
+        if (!shared_gate_up_proj || !shared_down_proj || !aligned16(shared_gate_up_proj) ||
+            !aligned16(shared_down_proj))
+            return MOE_ERR_INVALID_ARG;
+        if (wt == MOE_W_FP8_E4M3 && (!shared_gate_up_scale || !shared_down_scale ||
+                                     !aligned16(shared_gate_up_scale) || !aligned16(shared_down_scale)))
+            return MOE_ERR_INVALID_ARG;
+    }
+    if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    SharedSet sh;
+    sh.S = S;
+    sh.gate_up = shared_gate_up_proj;
+    sh.down = shared_down_proj;
+    sh.gate_up_scale = shared_gate_up_scale;
+    sh.down_scale = shared_down_scale;
+    if (shared_decode_serves(T, H, F, top_k, S, wt)) {
+        const DecodeWorkspace D = decode_workspace(T, H, F, E + S, top_k + S, wt);
+        if (!workspace || workspace_bytes < D.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+            return MOE_ERR_WORKSPACE;
+        return from_cuda(launch_decode_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                            top_k_weights, T, H, F, E, top_k, wsb, D, out, st, sh,
+                                            residual));
+    }
+    const SharedLayout SL = shared_workspace(T, H, F, E, top_k, S, wt);
+    if (!workspace || workspace_bytes < SL.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return MOE_ERR_WORKSPACE;
+    int32_t *idx2 = reinterpret_cast<int32_t *>(wsb + SL.idx2);
+    float *w2 = reinterpret_cast<float *>(wsb + SL.w2);
+    const cudaError_t e = launch_widen_routing(top_k_index, top_k_weights, T, E, top_k, S, idx2, w2, st);
+    if (e != cudaSuccess) return from_cuda(e);
+    // E4M3 tile height: the rule of the routed-only call (the shared experts
+    // add S experts of T rows each, one 16-row tile for T <= 16)
+    return run_prefill(hidden_states, gate_up_proj, down_proj, idx2, w2, top_k + S, T, H, F, E + S,
+                       wt, gate_up_scale, down_scale, out, workspace, SL.L.total, st,
+                       wt == MOE_W_FP8_E4M3 && fp8_decode_sized(T, top_k) ? kBNFp8Decode : kBNFp8,
+                       sh, residual);
 }
 
 moe_status_t moe_route_sigmoid_grouped(const float *logits, const float *bias, int T, int E,

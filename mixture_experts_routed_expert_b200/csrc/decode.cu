@@ -10,6 +10,9 @@
 //              stream row j of every touched down projection once, y_s =
 //              D_e[j] . h[s] for the slots of e, then
 //              out[t, j] = bf16( sum_{k in order} w[t,k] * y_{t*K+k} ).
+// Optional shared experts (S of them, weight 1) take slots K..K+S-1 of every
+// token after its K routed slots, with their own weight tensors, and an
+// optional residual is added after the slot sum.
 // D2 is launched as a programmatic dependent of D1: before waiting for D1 it
 // prefetches its own down-projection rows into L2, so both kernels stream
 // weights from HBM at the same time.  No atomics; fixed summation order.
@@ -24,10 +27,12 @@ constexpr int kUpWarps = 16;
 constexpr int kDownWarps = 16;
 constexpr int kSlotGroup = 1;   // slots of one expert handled per pass over the loaded rows
 
-// Distinct experts of the T*K slots, in order of first appearance, with the
-// slots of each in ascending order.  Built cooperatively by the first
-// kDecodeMaxSlots threads of the block (one slot each); every thread must call
-// it (it contains __syncthreads).
+// Distinct experts of the T*(K+S) slots, in order of first appearance, with
+// the slots of each in ascending order.  Slot t*(K+S)+k holds routed id
+// idx[t,k] for k < K (-1 when outside [0, E)) and shared expert E+(k-K)
+// after that.  Built cooperatively by the first kDecodeMaxSlots threads of the
+// block (one slot each); every thread must call it (it contains
+// __syncthreads).
 struct Touched {
     int n;
     int expert[kDecodeMaxSlots];
@@ -37,12 +42,20 @@ struct Touched {
     int u_of[kDecodeMaxSlots];     // touched index of each slot
 };
 
-__device__ void build_touched(const int32_t *__restrict__ idx, int TK, int E, Touched &u) {
+__device__ void build_touched(const int32_t *__restrict__ idx, int T, int K, int S, int E,
+                              Touched &u) {
     __shared__ int is_first[kDecodeMaxSlots];
+    const int K2 = K + S;
+    const int TK = T * K2;
     const int s = threadIdx.x;
     if (s < TK) {
-        const int e = __ldg(idx + s);
-        u.e_of[s] = (e >= 0 && e < E) ? e : -1;
+        const int t = s / K2, k = s - t * K2;
+        if (k < K) {
+            const int e = __ldg(idx + t * K + k);
+            u.e_of[s] = (e >= 0 && e < E) ? e : -1;
+        } else {
+            u.e_of[s] = E + (k - K);
+        }
     }
     __syncthreads();
     int e = -1, first = -1;
@@ -120,11 +133,15 @@ struct UpRows {
     uint4 g[VPL], u[VPL];
 };
 
-template <int VPL>
+template <int VPL, bool EXTRA>
 __device__ __forceinline__ void up_load(UpRows<VPL> &r, const uint4 *__restrict__ gate_up,
+                                        const uint4 *__restrict__ gate_up2, int E,
                                         const Touched &tu, int64_t it, int F, int nv, int lane) {
     const int ui = (int)(it / F), f = (int)(it - (int64_t)ui * F);
-    const uint4 *grow = gate_up + ((int64_t)tu.expert[ui] * 2 * F + f) * nv;
+    const int e = tu.expert[ui];
+    const uint4 *grow = (!EXTRA || e < E ? gate_up + (int64_t)e * 2 * F * nv
+                                         : gate_up2 + (int64_t)(e - E) * 2 * F * nv) +
+                        (int64_t)f * nv;
     const uint4 *urow = grow + (int64_t)F * nv;
 #pragma unroll
     for (int c = 0; c < VPL; ++c) {
@@ -158,12 +175,14 @@ __device__ __forceinline__ void up_compute(const UpRows<VPL> &r, const uint4 *__
     }
 }
 
-template <int VPL>
+template <int VPL, bool EXTRA>
 __global__ void __launch_bounds__(kUpWarps * 32, 1) decode_up_bf16(
-    const uint4 *__restrict__ x, const uint4 *__restrict__ gate_up, const int32_t *__restrict__ idx,
-    int T, int H, int F, int E, int K, __nv_bfloat16 *__restrict__ h) {
+    const uint4 *__restrict__ x, const uint4 *__restrict__ gate_up,
+    const uint4 *__restrict__ gate_up2, const int32_t *__restrict__ idx, int T, int H, int F, int E,
+    int K, int S_arg, __nv_bfloat16 *__restrict__ h) {
     __shared__ Touched tu;
-    build_touched(idx, T * K, E, tu);
+    const int S = EXTRA ? S_arg : 0;   // EXTRA = false: the routed-only form
+    build_touched(idx, T, K, S, E, tu);
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int nv = H / 8;
@@ -171,36 +190,49 @@ __global__ void __launch_bounds__(kUpWarps * 32, 1) decode_up_bf16(
     const int64_t i0 = items * blockIdx.x / gridDim.x, i1 = items * (blockIdx.x + 1) / gridDim.x;
     UpRows<VPL> ra, rb;
     int64_t it = i0 + warp;
-    if (it < i1) up_load(ra, gate_up, tu, it, F, nv, lane);
+    const int K2 = K + S;
+    if (it < i1) up_load<VPL, EXTRA>(ra, gate_up, gate_up2, E, tu, it, F, nv, lane);
     for (; it < i1; it += 2 * kUpWarps) {
         const int64_t nb = it + kUpWarps, na = it + 2 * kUpWarps;
-        if (nb < i1) up_load(rb, gate_up, tu, nb, F, nv, lane);
-        up_compute(ra, x, tu, it, F, K, nv, lane, h);
-        if (na < i1) up_load(ra, gate_up, tu, na, F, nv, lane);
-        if (nb < i1) up_compute(rb, x, tu, nb, F, K, nv, lane, h);
+        if (nb < i1) up_load<VPL, EXTRA>(rb, gate_up, gate_up2, E, tu, nb, F, nv, lane);
+        up_compute(ra, x, tu, it, F, K2, nv, lane, h);
+        if (na < i1) up_load<VPL, EXTRA>(ra, gate_up, gate_up2, E, tu, na, F, nv, lane);
+        if (nb < i1) up_compute(rb, x, tu, nb, F, K2, nv, lane, h);
     }
 }
 
 // D2.  Block b owns hidden rows [j0, j1).  One item = (row j, touched expert
 // u); a warp loads the down rows of two items before using either.  The
 // per-slot results y_s land in shared memory; after a block barrier,
-// out[t, j] = bf16( sum_{k in order} w[t,k] * y_{t*K+k} ).
-template <int VPL>
+// out[t, j] = bf16( sum_{k in order} w[t,k] * y_{t*K+k} [+ residual[t, j]] )
+// with weight 1 for the shared slots.  EXTRA = false compiles the routed-only
+// form (S = 0, no residual), whose registers fit the two-blocks-per-SM bound.
+template <int VPL, bool EXTRA>
 __global__ void __launch_bounds__(kDownWarps * 32, VPL <= 4 ? 2 : 1) decode_down_bf16(
-    const uint4 *__restrict__ down, const uint4 *__restrict__ h, const int32_t *__restrict__ idx,
-    const float *__restrict__ w, int T, int H, int F, int E, int K, __nv_bfloat16 *__restrict__ out) {
+    const uint4 *__restrict__ down, const uint4 *__restrict__ down2, const uint4 *__restrict__ h,
+    const int32_t *__restrict__ idx, const float *__restrict__ w, int T, int H, int F, int E, int K,
+    int S_arg, const __nv_bfloat16 *__restrict__ residual, __nv_bfloat16 *__restrict__ out) {
     __shared__ Touched tu;
-    extern __shared__ float ys[];     // [rows of this block][T*K]
-    build_touched(idx, T * K, E, tu);
+    __shared__ const uint4 *dbase[kDecodeMaxSlots];   // row j0 of each touched down projection
+    extern __shared__ float ys[];     // [rows of this block][T*(K+S)]
+    const int S = EXTRA ? S_arg : 0;
+    build_touched(idx, T, K, S, E, tu);
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int nv = F / 8;
-    const int TK = T * K;
+    const int K2 = K + S;
+    const int TK = T * K2;
     const int j0 = (int)((int64_t)H * blockIdx.x / gridDim.x);
     const int j1 = (int)((int64_t)H * (blockIdx.x + 1) / gridDim.x);
     // Stream this block's down rows into L2 while D1 is still running.
-    if (j1 > j0 && threadIdx.x < tu.n)
-        prefetch_l2_bulk(down + ((int64_t)tu.expert[threadIdx.x] * H + j0) * nv,
-                         (uint32_t)((j1 - j0) * F * 2));
+    if (threadIdx.x < tu.n) {
+        const int e = tu.expert[threadIdx.x];
+        const uint4 *b = (!EXTRA || e < E ? down + (int64_t)e * H * nv
+                                          : down2 + (int64_t)(e - E) * H * nv) +
+                         (int64_t)j0 * nv;
+        if (EXTRA) dbase[threadIdx.x] = b;
+        if (j1 > j0) prefetch_l2_bulk(b, (uint32_t)((j1 - j0) * F * 2));
+    }
+    if (EXTRA) __syncthreads();
     pdl_wait();
     const int items = (j1 - j0) * tu.n;
     for (int i = 2 * warp; i < items; i += 2 * kDownWarps) {
@@ -209,7 +241,9 @@ __global__ void __launch_bounds__(kDownWarps * 32, VPL <= 4 ? 2 : 1) decode_down
         for (int p = 0; p < 2; ++p) {
             const int it = i + p;
             const int jl = it / max(tu.n, 1), ui = it - jl * tu.n;
-            const uint4 *drow = down + ((int64_t)tu.expert[it < items ? ui : 0] * H + j0 + jl) * nv;
+            const int ue = it < items ? ui : 0;
+            const uint4 *drow = EXTRA ? dbase[ue] + (int64_t)jl * nv
+                                      : down + ((int64_t)tu.expert[ue] * H + j0 + jl) * nv;
 #pragma unroll
             for (int c = 0; c < VPL; ++c) {
                 const int v = c * 32 + lane;
@@ -249,11 +283,16 @@ __global__ void __launch_bounds__(kDownWarps * 32, VPL <= 4 ? 2 : 1) decode_down
     for (int q = threadIdx.x; q < (j1 - j0) * T; q += blockDim.x) {
         const int jl = q / T, t = q - jl * T;
         float acc = 0.f;
-        for (int k = 0; k < K; ++k) {
-            const int s = t * K + k;
+        for (int k = 0; k < K2; ++k) {
+            const int s = t * K2 + k;
             if (tu.e_of[s] < 0) continue;
-            acc = fmaf(w[s], ys[jl * TK + s], acc);
+            if (!EXTRA || k < K)
+                acc = fmaf(w[t * K + k], ys[jl * TK + s], acc);
+            else
+                acc += ys[jl * TK + s];
         }
+        if (EXTRA && residual != nullptr)
+            acc += __bfloat162float(residual[(int64_t)t * H + j0 + jl]);
         out[(int64_t)t * H + j0 + jl] = __float2bfloat16_rn(acc);
     }
 }
@@ -263,14 +302,19 @@ __global__ void __launch_bounds__(kDownWarps * 32, VPL <= 4 ? 2 : 1) decode_down
 cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *down,
                                const int32_t *idx, const float *w, int T, int H, int F, int E,
                                int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
-                               cudaStream_t st) {
+                               cudaStream_t st, const SharedSet &sh, const void *residual) {
     __nv_bfloat16 *h = (__nv_bfloat16 *)(ws + L.h);
+    const int S = sh.S;
+    const uint4 *gu2 = (const uint4 *)(S > 0 ? sh.gate_up : gate_up);
+    const uint4 *dn2 = (const uint4 *)(S > 0 ? sh.down : down);
     const int vpl_up = (H / 8 + 31) / 32, vpl_dn = (F / 8 + 31) / 32;
     int grid = num_sms();
     const dim3 blk(kUpWarps * 32);
     cudaError_t err;
-#define MOE_UP(V) launch_k(decode_up_bf16<V>, dim3(grid), blk, 0, st, false, (const uint4 *)x, \
-                           (const uint4 *)gate_up, idx, T, H, F, E, K, h)
+    const bool extra = S > 0 || residual != nullptr;
+#define MOE_UP(V)                                                                                 \
+    launch_k(extra ? decode_up_bf16<V, true> : decode_up_bf16<V, false>, dim3(grid), blk, 0, st, \
+             false, (const uint4 *)x, (const uint4 *)gate_up, gu2, idx, T, H, F, E, K, S, h)
     switch (vpl_up) {
         case 1: err = MOE_UP(1); break;
         case 2: err = MOE_UP(2); break;
@@ -285,10 +329,11 @@ cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *d
 #undef MOE_UP
     if (err != cudaSuccess) return err;
     grid = (vpl_dn <= 4 ? 2 : 1) * num_sms();
-    const size_t smem = sizeof(float) * ((H + grid - 1) / grid + 1) * T * K;
-#define MOE_DN(V) launch_k(decode_down_bf16<V>, dim3(grid), dim3(kDownWarps * 32), smem, st, true, \
-                           (const uint4 *)down, (const uint4 *)h, idx, w, T, H, F, E, K,        \
-                           (__nv_bfloat16 *)out)
+    const size_t smem = sizeof(float) * ((H + grid - 1) / grid + 1) * T * (K + S);
+#define MOE_DN(V)                                                                                \
+    launch_k(extra ? decode_down_bf16<V, true> : decode_down_bf16<V, false>, dim3(grid),           \
+             dim3(kDownWarps * 32), smem, st, true, (const uint4 *)down, dn2, (const uint4 *)h, idx, \
+             w, T, H, F, E, K, S, (const __nv_bfloat16 *)residual, (__nv_bfloat16 *)out)
     switch (vpl_dn) {
         case 1: return MOE_DN(1);
         case 2: return MOE_DN(2);

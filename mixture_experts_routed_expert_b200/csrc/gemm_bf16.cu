@@ -55,6 +55,7 @@ struct GemmArgs {
     const int32_t *offsets;      // [E+1] first routed row of each expert
     const int32_t *tiles;        // [E+1] prefix sum of row tiles per expert
     int E, MT, KB;               // experts, weight-row tiles per expert, k-blocks
+    int E_split;                 // experts >= E_split read the second weight map (shared set)
     int a_rows_per_expert;       // 2F (gate_up) or H (down)
     int up_offset;               // F: row offset of the up half (gate_up)
     __nv_bfloat16 *h;            // gate_up output [N][F]
@@ -68,8 +69,8 @@ struct GemmArgs {
 
 template <bool GATE_UP>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const GemmArgs args) {
+    grouped_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                      const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
     using C = Cfg<GATE_UP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
+        prefetch_tmap(&tmA2);
         prefetch_tmap(&tmB);
     }
     if (warp == 1) {
@@ -137,16 +139,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
                 const int nbox = (t.nrows + kBoxRows - 1) / kBoxRows;
                 const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * kBoxRows * 128;
-                const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
+                const bool second = t.e >= args.E_split;
+                const CUtensorMap *mA = second ? &tmA2 : &tmA;
+                const int arow = (second ? t.e - args.E_split : t.e) * args.a_rows_per_expert + t.m * kBM;
                 for (int kb = 0; kb < args.KB; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t *sA = ring + stage * C::STAGE_BYTES;
                     uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     armed[stage] = (int)phase;
-                    tma_load_2d(sA, &tmA, &full[stage], kb * kBK, arow, pol_w);
+                    tma_load_2d(sA, mA, &full[stage], kb * kBK, arow, pol_w);
                     if (GATE_UP)
-                        tma_load_2d(sA + C::A_BYTES, &tmA, &full[stage], kb * kBK,
+                        tma_load_2d(sA + C::A_BYTES, mA, &full[stage], kb * kBK,
                                     arow + args.up_offset, pol_w);
                     for (int b = 0; b < nbox; ++b)
                         tma_load_2d(sB + b * kBoxRows * 128, &tmB, &full[stage], kb * kBK,
@@ -274,7 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <bool GATE_UP>
-cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmArgs &args,
+cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &a2, const CUtensorMap &b,
+                       const GemmArgs &args,
                        cudaStream_t st) {
     using C = Cfg<GATE_UP>;
     const size_t smem = C::smem_bytes(args.E);
@@ -289,25 +294,35 @@ cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &b, const GemmArg
         attr_done[dev & 63] = 1;
     }
     return launch_k(grouped_gemm_bf16<GATE_UP>, dim3(num_sms()), dim3(kThreads), smem, st, true, a,
-                    b, args);
+                    a2, b, args);
 }
 
 }  // namespace
 
 cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float *topw, int64_t T,
                               int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
-                              cudaStream_t st) {
+                              cudaStream_t st, const SharedSet &sh) {
     const uint64_t N = (uint64_t)T * K;
-    CUtensorMap ta, tb, tc, td;
+    CUtensorMap ta, tb, tc, td, ta2, tc2;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    if (!make_tmap(&ta, BF, 2, gate_up, (uint64_t)E * 2 * F, H, kBM) ||
+    const int E_split = E - sh.S;  // routed experts; ids E_split.. are the shared set
+    if (!make_tmap(&ta, BF, 2, gate_up, (uint64_t)E_split * 2 * F, H, kBM) ||
         !make_tmap(&tb, BF, 2, ws + L.xperm, N, H, kBoxRows) ||
-        !make_tmap(&tc, BF, 2, down, (uint64_t)E * H, F, kBM) ||
+        !make_tmap(&tc, BF, 2, down, (uint64_t)E_split * H, F, kBM) ||
         !make_tmap(&td, BF, 2, ws + L.h, N, F, kBoxRows))
         return cudaErrorInvalidValue;
+    if (sh.S > 0) {
+        if (!make_tmap(&ta2, BF, 2, sh.gate_up, (uint64_t)sh.S * 2 * F, H, kBM) ||
+            !make_tmap(&tc2, BF, 2, sh.down, (uint64_t)sh.S * H, F, kBM))
+            return cudaErrorInvalidValue;
+    } else {
+        ta2 = ta;
+        tc2 = tc;
+    }
     GemmArgs g = {};
     g.offsets = (const int32_t *)(ws + L.offsets);
     g.E = E;
+    g.E_split = E_split;
     g.perm = (const int32_t *)(ws + L.perm);
     g.topw = topw;
     g.status = (int32_t *)(ws + L.status);
@@ -322,7 +337,7 @@ cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float
     a1.KB = H / kBK;
     a1.a_rows_per_expert = 2 * F;
     a1.up_offset = F;
-    cudaError_t err = launch_one<true>(ta, tb, a1, st);
+    cudaError_t err = launch_one<true>(ta, ta2, tb, a1, st);
     if (err != cudaSuccess) return err;
 
     GemmArgs a2 = g;
@@ -331,7 +346,7 @@ cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float
     a2.KB = F / kBK;
     a2.a_rows_per_expert = H;
     a2.up_offset = 0;
-    return launch_one<false>(tc, td, a2, st);
+    return launch_one<false>(tc, tc2, td, a2, st);
 }
 
 }  // namespace moe

@@ -69,8 +69,10 @@ struct Cfg8 {
 struct Gemm8Args {
     const int32_t *offsets, *tiles;
     int E, MT, KB;
+    int E_split;             // experts >= E_split read the second weight map and scales
     int a_rows_per_expert, up_offset;
-    const float *wscale;     // [E * rows][KB] weight scales
+    const float *wscale;     // [E_split * rows][KB] weight scales
+    const float *wscale2;    // [(E - E_split) * rows][KB] weight scales of the second set
     const float *xscale;     // [N][KB] activation scales of the routed rows
     uint8_t *hq;             // gate_up: [N][F] e4m3
     float *hs;               // gate_up: [N][F/128]
@@ -89,8 +91,8 @@ __device__ __forceinline__ void epi_sync() {
 
 template <bool GATE_UP, int BN>
 __global__ void __launch_bounds__(kThreads8, 1)
-    grouped_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const Gemm8Args args) {
+    grouped_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                     const __grid_constant__ CUtensorMap tmB, const Gemm8Args args) {
     using C = Cfg8<GATE_UP, BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
+        prefetch_tmap(&tmA2);
         prefetch_tmap(&tmB);
     }
     if (warp == 1) {
@@ -160,16 +163,18 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
                 const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
                 const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * C::BOX * 128;
-                const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
+                const bool second = t.e >= args.E_split;
+                const CUtensorMap *mA = second ? &tmA2 : &tmA;
+                const int arow = (second ? t.e - args.E_split : t.e) * args.a_rows_per_expert + t.m * kBM;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t *sA = ring + stage * C::STAGE_BYTES;
                     uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     armed[stage] = (int)phase;
-                    tma_load_2d(sA, &tmA, &full[stage], kb * 128, arow, pol_w);
+                    tma_load_2d(sA, mA, &full[stage], kb * 128, arow, pol_w);
                     if (GATE_UP)
-                        tma_load_2d(sA + C::A_BYTES, &tmA, &full[stage], kb * 128,
+                        tma_load_2d(sA + C::A_BYTES, mA, &full[stage], kb * 128,
                                     arow + args.up_offset, pol_w);
                     for (int b = 0; b < nbox; ++b)
                         tma_load_2d(sB + b * C::BOX * 128, &tmB, &full[stage], kb * 128,
@@ -241,7 +246,9 @@ __global__ void __launch_bounds__(kThreads8, 1)
             // Weight scales of the tile's 128 rows: with STAGE_SCALES they
             // arrive in shared memory SG k-blocks at a time, one group ahead
             // (asynchronous copies); otherwise each is read one k-block ahead.
-            const float *wsrc = args.wscale + ((size_t)t.e * args.a_rows_per_expert + t.m * kBM) * KB;
+            const bool second = t.e >= args.E_split;
+            const float *wsrc = (second ? args.wscale2 : args.wscale) +
+                                ((size_t)(second ? t.e - args.E_split : t.e) * args.a_rows_per_expert + t.m * kBM) * KB;
             const float *wsg = wsrc + (size_t)row * KB;
             const float *wsu = wsrc + (size_t)(row + args.up_offset) * KB;
             auto issue_scales = [&](int kb0, int buf) {
@@ -455,8 +462,8 @@ __global__ void __launch_bounds__(kThreads8, 1)
 }
 
 template <bool GATE_UP, int BN>
-cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &b, const Gemm8Args &args,
-                        cudaStream_t st) {
+cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &a2, const CUtensorMap &b,
+                        const Gemm8Args &args, cudaStream_t st) {
     using C = Cfg8<GATE_UP, BN>;
     static size_t attr_bytes[64] = {};          // per device: dynamic shared memory limit set so far
     int dev = 0;
@@ -474,7 +481,7 @@ cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &b, const Gemm8A
         attr_bytes[dev & 63] = need;
     }
     return launch_k(grouped_gemm_fp8<GATE_UP, BN>, dim3(num_sms()), dim3(kThreads8), need, st, true,
-                    a, b, a8);
+                    a, a2, b, a8);
 }
 
 }  // namespace
@@ -482,21 +489,31 @@ cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &b, const Gemm8A
 
 cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
                              const float *topw, int64_t T, int H, int F, int E, int K, int bn,
-                             uint8_t *ws, const Workspace &L, cudaStream_t st) {
+                             uint8_t *ws, const Workspace &L, cudaStream_t st, const SharedSet &sh) {
     if (H / 128 > kMaxKB8 || F / 128 > kMaxKB8) return cudaErrorInvalidValue;
     if (bn != kBNFp8 && bn != kBNFp8Decode) return cudaErrorInvalidValue;
     const int box = bn < 32 ? bn : 32;
     const uint64_t N = (uint64_t)T * K;
-    CUtensorMap ta, tb, tc, td;
+    CUtensorMap ta, tb, tc, td, ta2, tc2;
     const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    if (!make_tmap(&ta, U8, 1, w13, (uint64_t)E * 2 * F, H, kBM) ||
+    const int E_split = E - sh.S;  // routed experts; ids E_split.. are the shared set
+    if (!make_tmap(&ta, U8, 1, w13, (uint64_t)E_split * 2 * F, H, kBM) ||
         !make_tmap(&tb, U8, 1, ws + L.xperm, N, H, box) ||
-        !make_tmap(&tc, U8, 1, w2, (uint64_t)E * H, F, kBM) ||
+        !make_tmap(&tc, U8, 1, w2, (uint64_t)E_split * H, F, kBM) ||
         !make_tmap(&td, U8, 1, ws + L.h, N, F, box))
         return cudaErrorInvalidValue;
+    if (sh.S > 0) {
+        if (!make_tmap(&ta2, U8, 1, sh.gate_up, (uint64_t)sh.S * 2 * F, H, kBM) ||
+            !make_tmap(&tc2, U8, 1, sh.down, (uint64_t)sh.S * H, F, kBM))
+            return cudaErrorInvalidValue;
+    } else {
+        ta2 = ta;
+        tc2 = tc;
+    }
     Gemm8Args g = {};
     g.offsets = (const int32_t *)(ws + L.offsets);
     g.E = E;
+    g.E_split = E_split;
     g.perm = (const int32_t *)(ws + L.perm);
     g.topw = topw;
     g.status = (int32_t *)(ws + L.status);
@@ -513,6 +530,7 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     a1.a_rows_per_expert = 2 * F;
     a1.up_offset = F;
     a1.wscale = w13s;
+    a1.wscale2 = sh.S > 0 ? sh.gate_up_scale : w13s;
     a1.xscale = (const float *)(ws + L.xscale);
 
     Gemm8Args a2 = g;
@@ -522,15 +540,16 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     a2.a_rows_per_expert = H;
     a2.up_offset = 0;
     a2.wscale = w2s;
+    a2.wscale2 = sh.S > 0 ? sh.down_scale : w2s;
     a2.xscale = (const float *)(ws + L.hscale);
     if (bn == kBNFp8Decode) {
-        const cudaError_t err = launch_one8<true, kBNFp8Decode>(ta, tb, a1, st);
+        const cudaError_t err = launch_one8<true, kBNFp8Decode>(ta, ta2, tb, a1, st);
         if (err != cudaSuccess) return err;
-        return launch_one8<false, kBNFp8Decode>(tc, td, a2, st);
+        return launch_one8<false, kBNFp8Decode>(tc, tc2, td, a2, st);
     }
-    const cudaError_t err = launch_one8<true, kBNFp8>(ta, tb, a1, st);
+    const cudaError_t err = launch_one8<true, kBNFp8>(ta, ta2, tb, a1, st);
     if (err != cudaSuccess) return err;
-    return launch_one8<false, kBNFp8>(tc, td, a2, st);
+    return launch_one8<false, kBNFp8>(tc, tc2, td, a2, st);
 }
 
 }  // namespace moe

@@ -55,6 +55,16 @@ moe_status_t validate_forward(const void *x, const void *gu, const void *dn, con
 // True when T tokens x K slots are served by the decode kernels.
 bool decode_path_fits(int T, int K, int H, int F);
 
+// Always-active (shared) experts served as extra expert ids E_routed..E_routed+S-1
+// of the grouped GEMMs; their weights live in their own tensors.
+struct SharedSet {
+    int S = 0;                          // number of shared experts (0: none)
+    const void *gate_up = nullptr;      // [S][2F][H]
+    const void *down = nullptr;         // [S][H][F]
+    const float *gate_up_scale = nullptr;  // E4M3: [S][2F][H/128]
+    const float *down_scale = nullptr;     // E4M3: [S][H][F/128]
+};
+
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 int num_sms();
 
@@ -68,17 +78,26 @@ cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, con
                                  int32_t *perm, int32_t *inv, cudaStream_t st);
 cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float *topw, int64_t T,
                               int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
-                              cudaStream_t st);
+                              cudaStream_t st, const SharedSet &sh = SharedSet());
+// E counts the routed and the shared experts (sh.S of them, the last ids).
 // bn: kBNFp8 or kBNFp8Decode; must match the tile prefixes of the permutation.
 cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
                              const float *topw, int64_t T, int H, int F, int E, int K, int bn,
-                             uint8_t *ws, const Workspace &L, cudaStream_t st);
+                             uint8_t *ws, const Workspace &L, cudaStream_t st,
+                             const SharedSet &sh = SharedSet());
+// residual: optional [T][H] bf16 added after the slot sum (nullptr: none).
 cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, const uint8_t *ws,
-                           const Workspace &L, void *out, cudaStream_t st);
+                           const Workspace &L, void *out, cudaStream_t st,
+                           const void *residual = nullptr);
+// idx2/w2 [T][K+S]: the K routed slots (ids outside [0,E) -> -1), then the S
+// shared ids E..E+S-1 with weight 1.
+cudaError_t launch_widen_routing(const int32_t *idx, const float *w, int64_t T, int E, int K,
+                                 int S, int32_t *idx2, float *w2, cudaStream_t st);
 cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *down,
                                const int32_t *idx, const float *w, int T, int H, int F, int E,
                                int K, uint8_t *ws, const DecodeWorkspace &L, void *out,
-                               cudaStream_t st);
+                               cudaStream_t st, const SharedSet &sh = SharedSet(),
+                               const void *residual = nullptr);
 cudaError_t launch_quantize(const void *x, int64_t rows, int cols, void *xq, float *scale,
                             cudaStream_t st);
 cudaError_t launch_route(const float *logits, const float *bias, int64_t T, int E, int num_groups,

@@ -201,11 +201,39 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
     }
 }
 
-// S6: out[t, j] = bf16( sum_{k in order} y[t*K + k, j] ) over slots with a
-// valid expert id (y already holds w[t,k] * down_e(h)).  4 columns per thread.
+// Shared experts as extra slots: row t of the widened routing holds the K
+// routed ids (ids outside [0, E) become -1 so they can never name a shared
+// expert) followed by the S shared ids E..E+S-1 with weight 1.
+__global__ void __launch_bounds__(256) widen_routing_kernel(const int32_t *__restrict__ idx,
+                                                            const float *__restrict__ w, int64_t T,
+                                                            int E, int K, int S,
+                                                            int32_t *__restrict__ idx2,
+                                                            float *__restrict__ w2) {
+    pdl_wait();
+    const int K2 = K + S;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T * K2) return;
+    const int64_t t = i / K2;
+    const int k = (int)(i - t * K2);
+    if (k < K) {
+        const int e = idx[t * K + k];
+        idx2[i] = e >= 0 && e < E ? e : -1;
+        w2[i] = w[t * K + k];
+    } else {
+        idx2[i] = E + (k - K);
+        w2[i] = 1.0f;
+    }
+    pdl_launch_dependents();
+}
+
+// S6: out[t, j] = bf16( sum_{k in order} y[t*K + k, j] [+ residual[t, j]] )
+// over slots with a valid expert id (y already holds w[t,k] * down_e(h)); the
+// residual, when given, is added after the slot sum.  4 columns per thread.
 __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__ y,
                                                       const int32_t *__restrict__ idx, int64_t T,
-                                                      int H, int E, int K, uint2 *__restrict__ out) {
+                                                      int H, int E, int K,
+                                                      const uint2 *__restrict__ residual,
+                                                      uint2 *__restrict__ out) {
     pdl_wait();
     const int nv = H / 4;
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -234,6 +262,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
                 acc.x += a[i].x; acc.y += a[i].y; acc.z += a[i].z; acc.w += a[i].w;
             }
         }
+    }
+    if (residual != nullptr) {
+        const uint2 r = __ldg(residual + t * nv + v);
+        acc.x += bf16_lo(r.x); acc.y += bf16_hi(r.x); acc.z += bf16_lo(r.y); acc.w += bf16_hi(r.y);
     }
     uint2 o;
     o.x = pack_bf16x2(acc.x, acc.y);
@@ -305,10 +337,18 @@ cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, con
 }
 
 cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, const uint8_t *ws,
-                           const Workspace &L, void *out, cudaStream_t st) {
+                           const Workspace &L, void *out, cudaStream_t st, const void *residual) {
     const int64_t n = T * (H / 4);
     return launch_k(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, true,
-                    (const float4 *)(ws + L.y), idx, T, H, E, K, (uint2 *)out);
+                    (const float4 *)(ws + L.y), idx, T, H, E, K, (const uint2 *)residual,
+                    (uint2 *)out);
+}
+
+cudaError_t launch_widen_routing(const int32_t *idx, const float *w, int64_t T, int E, int K,
+                                 int S, int32_t *idx2, float *w2, cudaStream_t st) {
+    const int64_t n = T * (K + S);
+    return launch_k(widen_routing_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, true,
+                    idx, w, T, E, K, S, idx2, w2);
 }
 
 }  // namespace moe

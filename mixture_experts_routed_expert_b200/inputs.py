@@ -143,6 +143,25 @@ def fp8_layer(T: int, seed: int = 0, device="cpu", zipf: Optional[float] = None,
     return Fp8Layer(x, w13, w13s, w2, w2s, logits, bias, dict(T=T, H=H, F=F, E=E))
 
 
+def shared_experts_bf16(S: int, H: int, F: int, seed: int = 0, device="cpu"):
+    """S always-active experts: (gate_up [S,2F,H], down [S,H,F]) bf16, same
+    init scale as the routed experts."""
+    g = _gen(seed + 2000003, device)
+    gu = (torch.randn(S, 2 * F, H, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    dn = (torch.randn(S, H, F, generator=g, device=device) * 0.02).to(torch.bfloat16)
+    return gu, dn
+
+
+def shared_experts_fp8(S: int, H: int, F: int, seed: int = 0, device="cpu"):
+    """S always-active E4M3 experts: (w13, w13_scale, w2, w2_scale)."""
+    return fp8_weights(seed + 3000017, device, H, F, S)
+
+
+def residual_bf16(T: int, H: int, seed: int = 0, device="cpu"):
+    g = _gen(seed + 4000037, device)
+    return torch.randn(T, H, generator=g, device=device).to(torch.bfloat16)
+
+
 # --- host views for the oracle (numpy bit patterns) -------------------------
 
 def bf16_bits(t: torch.Tensor):

@@ -66,3 +66,31 @@ def test_host_validation_without_gpu(mod):
     # quantiser limits
     assert L.quantize_fp8_block128(p, 4, 100, p, p, N) == 1
     assert L.quantize_fp8_block128(p, 0, 128, p, p, N) == 0
+
+
+def test_shared_entry_host_checks(mod):
+    """moe_experts_with_shared: sizes, workspace and pointer checks on the host."""
+    ws = mod.moe_experts_shared_workspace_size
+    # widened to E+S experts and K+S slots, plus the widened routing
+    assert ws(64, 1280, 896, 64, 6, 2) > mod.moe_experts_workspace_size(64, 1280, 896, 66, 8)
+    assert ws(64, 1280, 896, 64, 6, 0) > mod.moe_experts_workspace_size(64, 1280, 896, 64, 6)
+    assert ws(64, 1280, 896, 64, 6, 11) == 0       # K + S > 16
+    assert ws(64, 1280, 896, 1020, 6, 5) == 0      # E + S > 1024
+    assert ws(64, 1280, 896, 64, 6, -1) == 0
+    L = mod.lib
+    N = None
+    p = ctypes.c_void_p(0x1000)
+    q = ctypes.c_void_p(0x1001)
+    big = 1 << 34
+    f = L.moe_experts_with_shared
+    # T == 0 no-op; bad S
+    assert f(N, N, N, N, N, 6, 0, 1280, 896, 64, 0, N, N, N, N, N, N, 2, N, N, N, 0, N) == 0
+    assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, p, p, N, N, 11, N, p, p, big, N) == 1
+    # shared weights missing or misaligned; residual misaligned
+    assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, N, p, N, N, 2, N, p, p, big, N) == 1
+    assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, q, p, N, N, 2, N, p, p, big, N) == 1
+    assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, p, p, N, N, 2, q, p, p, big, N) == 1
+    # E4M3 without the shared scales
+    assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 1, p, p, p, p, N, N, 2, N, p, p, big, N) == 1
+    # workspace too small
+    assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, p, p, N, N, 2, N, p, p, 4096, N) == 3
