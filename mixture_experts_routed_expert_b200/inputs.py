@@ -143,6 +143,75 @@ def fp8_layer(T: int, seed: int = 0, device="cpu", zipf: Optional[float] = None,
     return Fp8Layer(x, w13, w13s, w2, w2s, logits, bias, dict(T=T, H=H, F=F, E=E))
 
 
+# --- MXFP4 routed weights (offline weight preparation) ----------------------
+
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)   # codes 0..7; bit 3 = sign
+
+
+def e2m1_codes(v: torch.Tensor) -> torch.Tensor:
+    """Nearest E2M1 code of each value (ties to the even code, i.e. the even
+    mantissa), magnitudes above 6 saturate to 6.  Returns uint8 codes 0..15."""
+    a = v.abs()
+    # midpoints between neighbouring magnitudes; a tie goes to the even code
+    mids = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+    code = torch.zeros_like(a, dtype=torch.uint8)
+    for i, m in enumerate(mids):
+        upper_even = (i + 1) % 2 == 0          # code i+1 has an even mantissa
+        code = code + ((a > m) | ((a == m) & upper_even)).to(torch.uint8)
+    return code | ((v < 0).to(torch.uint8) << 3)
+
+
+def pack_e2m1(codes: torch.Tensor) -> torch.Tensor:
+    """[..., C] codes -> [..., C/2] bytes, even column in the low nibble."""
+    return codes[..., 0::2] | (codes[..., 1::2] << 4)
+
+
+def block_scale_layout(sc: torch.Tensor) -> torch.Tensor:
+    """E8M0 scales [..., R, C/32] -> the tensor-core block layout, flattened
+    over (R, C/32): one 512-byte block per 128 rows x 128 columns, blocks in
+    [R/128][C/128] order, scale (r, c) at byte (r%32)*16 + ((r%128)//32)*4 +
+    (c%128)//32 of its block."""
+    *lead, R, C32 = sc.shape
+    t = sc.reshape(*lead, R // 128, 4, 32, C32 // 4, 4)       # (rb, m1, m0, cb, j)
+    n = len(lead)
+    perm = list(range(n)) + [n, n + 3, n + 2, n + 1, n + 4]    # (rb, cb, m0, m1, j)
+    return t.permute(*perm).contiguous().reshape(*lead, R * C32)
+
+
+def quantize_weight_mxf4(wf: torch.Tensor):
+    """Offline MXFP4 quantisation of [..., R, C] fp32 weights (OCP
+    Microscaling): per (row, 32 columns) the shared exponent
+    X = floor(log2(amax)) - 2 (E2M1's largest exponent), clamped to
+    [-127, 127] (-127 for an all-zero block), elements E2M1(w / 2^X).
+    Returns (packed codes [..., R, C/2] uint8, E8M0 scales in the block
+    layout [..., R*C/32] uint8)."""
+    *lead, R, C = wf.shape
+    blk = wf.reshape(*lead, R, C // 32, 32)
+    amax = blk.abs().amax(dim=-1)
+    X = torch.where(amax > 0, torch.floor(torch.log2(torch.where(amax > 0, amax, torch.ones_like(amax)))) - 2,
+                    torch.full_like(amax, -127.0)).clamp(-127, 127)
+    codes = e2m1_codes(blk / torch.exp2(X).unsqueeze(-1)).reshape(*lead, R, C)
+    return pack_e2m1(codes), block_scale_layout((X + 127).to(torch.uint8))
+
+
+def mxf4_weights(seed: int = 0, device="cpu", H=None, F=None, E=None):
+    """DeepSeek-V3-like experts with MXFP4 weights: (w13 [E,2F,H/2],
+    w13_sc [E,2F*H/32], w2 [E,H,F/2], w2_sc [E,H*F/32]), weights drawn fp32
+    ~ N(0, 0.02^2) expert by expert, as for the E4M3 layer."""
+    H = H or DSV3_FP8["H"]; F = F or DSV3_FP8["F"]; E = E or DSV3_FP8["E"]
+    g = _gen(seed + 5000011, device)
+    w13 = torch.empty(E, 2 * F, H // 2, dtype=torch.uint8, device=device)
+    w13s = torch.empty(E, 2 * F * H // 32, dtype=torch.uint8, device=device)
+    w2 = torch.empty(E, H, F // 2, dtype=torch.uint8, device=device)
+    w2s = torch.empty(E, H * F // 32, dtype=torch.uint8, device=device)
+    for e in range(E):
+        q, sc = quantize_weight_mxf4(torch.randn(2 * F, H, generator=g, device=device) * 0.02)
+        w13[e].copy_(q); w13s[e].copy_(sc)
+        q, sc = quantize_weight_mxf4(torch.randn(H, F, generator=g, device=device) * 0.02)
+        w2[e].copy_(q); w2s[e].copy_(sc)
+    return w13, w13s, w2, w2s
+
+
 def shared_experts_bf16(S: int, H: int, F: int, seed: int = 0, device="cpu"):
     """S always-active experts: (gate_up [S,2F,H], down [S,H,F]) bf16, same
     init scale as the routed experts."""

@@ -44,10 +44,13 @@ def lib():
                                                      i32, P, P]
         L.oracle_moe_forward_shared_fp8.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, P,
                                                     P, P, P, i32, P, P]
+        L.oracle_mxf4_dequant.argtypes = [P, P, i64, i64, P]
+        L.oracle_moe_forward_mxf4.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, P]
         L.oracle_num_threads.restype = ctypes.c_int
         for fn in ("oracle_bf16_from_f64", "oracle_e4m3_from_f64", "oracle_e4m3_to_f64",
                    "oracle_quantize_fp8_block128", "oracle_route_sigmoid_grouped",
-                   "oracle_permute", "oracle_moe_forward_bf16", "oracle_moe_forward_fp8"):
+                   "oracle_permute", "oracle_moe_forward_bf16", "oracle_moe_forward_fp8",
+                   "oracle_mxf4_dequant", "oracle_moe_forward_mxf4"):
             getattr(L, fn).restype = None
         _lib = L
     return _lib
@@ -223,4 +226,38 @@ def moe_forward_shared_fp8(x, w13, w13_scale, w2, w2_scale, idx, w, sw13, sw13_s
     out = np.empty((T, H), np.uint16)
     lib().oracle_moe_forward_shared_fp8(px, pa, psa, pb, psb, pi, pw, T, H, F2 // 2, E, ix.shape[1],
                                         pc, psc, pdd, psd, S, pr, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def mxf4_dequant(q, sc, R, C):
+    """Packed MXFP4 matrix -> fp64 [R, C]: q [R, C/2] bytes (even column in the
+    low nibble), sc the E8M0 scales in the tensor-core block layout (one
+    512-byte block per 128 x 128, byte (r%32)*16 + ((r%128)//32)*4 + (c%128)//32)."""
+    q, pq = _c(q, np.uint8)
+    sc, ps = _c(sc, np.uint8)
+    assert q.size == R * C // 2 and sc.size == R * C // 32
+    out = np.empty((R, C), np.float64)
+    lib().oracle_mxf4_dequant(pq, ps, R, C, out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def moe_forward_mxf4(x, w13, w13_sc, w2, w2_sc, idx, w):
+    """MXFP4 routed weights (w13 [E,2F,H/2], w2 [E,H,F/2] packed E2M1; scales
+    E8M0 in the block layout, 2F*H/32 and H*F/32 bytes per expert), FP8
+    activations (block-128 E4M3 rule).  Returns out [T,H] bf16 bits."""
+    x, px = _c(x, np.uint16)
+    a, pa = _c(w13, np.uint8)
+    sa, psa = _c(w13_sc, np.uint8)
+    b, pb = _c(w2, np.uint8)
+    sb, psb = _c(w2_sc, np.uint8)
+    ix, pi = _c(idx, np.int32)
+    ww, pw = _c(w, np.float32)
+    T, H = x.shape
+    E, F2 = a.shape[0], a.shape[1]
+    F = F2 // 2
+    assert a.shape == (E, F2, H // 2) and b.shape == (E, H, F // 2)
+    assert sa.size == E * F2 * H // 32 and sb.size == E * H * F // 32
+    out = np.empty((T, H), np.uint16)
+    lib().oracle_moe_forward_mxf4(px, pa, psa, pb, psb, pi, pw, T, H, F, E, ix.shape[1],
+                                  out.ctypes.data_as(ctypes.c_void_p))
     return out

@@ -22,6 +22,10 @@
  *    bf16_to_fp8_quantize (block 128, E4M3 + power-of-two scale),
  *    moe_w13_fp8_layer / moe_w2_fp8_layer (per (row,128-col) fp32 weight
  *    scales), moe_silu_mul_layer, moe_local_reduction (weighted sum over k).
+ *  - GC MoE issue on the DeepGEMM tracker (FP8 activations with packed FP4
+ *    routed weights), the DeepGEMM Mega MoE news page (FP8 x FP4) and the
+ *    sgl-deep-gemm commit list ("MXF4 kind"): the MXFP4 weight format of
+ *    the OCP Microscaling spec (E2M1 elements, one E8M0 scale per 32).
  *
  * Parity pins: every exported function is pinned by tests under tests/
  * (test_oracle_*.py) against library routines, closed forms, invariants and
@@ -411,6 +415,118 @@ void oracle_moe_forward_fp8(const uint16_t *x, const uint8_t *w13, const float *
                             const float *w, int64_t T, int H, int F, int E, int K, uint16_t *out) {
     oracle_moe_forward_shared_fp8(x, w13, w13_scale, w2, w2_scale, idx, w, T, H, F, E, K, NULL, NULL,
                                   NULL, NULL, 0, NULL, out);
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP4 (MXFP4) routed weights with FP8 activations                          */
+/* ("Supporting MegaKernel ..." / GC MoE issue: FP8 activations x packed FP4 */
+/* routed weights; DeepGEMM Mega MoE news: FP8 x FP4; sgl-deep-gemm commit    */
+/* list: "MXF4 kind")                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* OCP Microscaling FP4, E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0
+ * mantissa.  Exponent field 0 is subnormal: 0.5 * mantissa; otherwise
+ * 2^(e-1) * (1 + mantissa/2).  Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static double e2m1_value(unsigned nib) {
+    unsigned e = (nib >> 1) & 3u, m = nib & 1u;
+    double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, (int)e - 1);
+    return (nib & 8u) ? -mag : mag;
+}
+
+/* OCP E8M0 block scale: 2^(b - 127); b = 255 encodes NaN. */
+static double e8m0_value(uint8_t b) { return b == 255 ? NAN : ldexp(1.0, (int)b - 127); }
+
+/* Element (r, c) of a packed MXFP4 matrix with R rows and C columns
+ * (C % 128 == 0, R % 128 == 0):
+ *   q  [R][C/2] bytes: element c of a row in byte c/2, even c in the low
+ *      nibble, odd c in the high nibble;
+ *   sc block-scale bytes (E8M0, one per row and 32 columns) in the tensor
+ *      core's block layout: one 512-byte block per (128 rows, 128 columns),
+ *      blocks ordered [R/128][C/128], and inside a block the scale of
+ *      (r, c) at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 128) / 32.
+ * Value = e2m1(code) * 2^(scale - 127). */
+static int64_t mxf4_scale_index(int64_t r, int64_t c, int64_t C) {
+    int64_t blk = (r / 128) * (C / 128) + c / 128;
+    return blk * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 128) / 32;
+}
+static double mxf4_element(const uint8_t *q, const uint8_t *sc, int64_t C, int64_t r, int64_t c) {
+    uint8_t byte = q[r * (C / 2) + c / 2];
+    unsigned nib = (c & 1) ? (unsigned)(byte >> 4) : (unsigned)(byte & 15u);
+    return e2m1_value(nib) * e8m0_value(sc[mxf4_scale_index(r, c, C)]);
+}
+
+/* Dequantise a packed MXFP4 matrix (layout above) to fp64 [R][C]. */
+void oracle_mxf4_dequant(const uint8_t *q, const uint8_t *sc, int64_t R, int64_t C, double *out) {
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c) out[r * C + c] = mxf4_element(q, sc, C, r, c);
+}
+
+/* One expert's contribution for one token with MXFP4 weights:
+ * W13 [2F][H/2] + S13 (blocks of the [2F, H] matrix), W2 [H][F/2] + S2
+ * (blocks of [H, F]); xd = the token's block-128 E4M3 activations,
+ * dequantised.  h = bf16(SiLU(g) u) is quantised per 128 features by the
+ * block-128 E4M3 rule and dequantised before the down projection (the same
+ * activation path as the FP8 layers).  Scratch: wr [max(H,F)], hv, hd [F],
+ * hq [F], hs [F/128]. */
+static void contrib_mxf4(const double *xd, const uint8_t *W13, const uint8_t *S13, const uint8_t *W2,
+                         const uint8_t *S2, int H, int F, double wk, double *wr, double *hv,
+                         double *hd, uint8_t *hq, float *hs, double *acc) {
+    int fb_n = F / 128;
+    for (int f = 0; f < F; ++f) {
+        double g = 0.0, u = 0.0;
+        for (int i = 0; i < H; ++i) wr[i] = mxf4_element(W13, S13, H, f, i);
+        for (int i = 0; i < H; ++i) g += wr[i] * xd[i];
+        for (int i = 0; i < H; ++i) wr[i] = mxf4_element(W13, S13, H, (int64_t)F + f, i);
+        for (int i = 0; i < H; ++i) u += wr[i] * xd[i];
+        hv[f] = bf16_value(bf16_from_double(silu(g) * u));
+    }
+    quantize_blocks(hv, fb_n, hq, hs);
+    for (int f = 0; f < F; ++f) hd[f] = e4m3_value(hq[f]) * (double)hs[f / 128];
+    for (int j = 0; j < H; ++j) {
+        double y = 0.0;
+        for (int f = 0; f < F; ++f) wr[f] = mxf4_element(W2, S2, F, j, f);
+        for (int f = 0; f < F; ++f) y += wr[f] * hd[f];
+        acc[j] += wk * y;
+    }
+}
+
+/* MXFP4 routed weights, FP8 activations:
+ *   w13 [E][2F][H/2] packed E2M1 + w13_sc (E8M0 blocks of each expert's
+ *   [2F, H] matrix, 2F*H/32 bytes per expert), w2 [E][H][F/2] + w2_sc
+ *   (H*F/32 bytes per expert), layouts as for mxf4_element.
+ * x (bf16) is quantised per 128 columns by the block-128 E4M3 rule; every
+ * operand is dequantised before the fp64 dot products; out = bf16(sum_k w y). */
+void oracle_moe_forward_mxf4(const uint16_t *x, const uint8_t *w13, const uint8_t *w13_sc,
+                             const uint8_t *w2, const uint8_t *w2_sc, const int32_t *idx,
+                             const float *w, int64_t T, int H, int F, int E, int K, uint16_t *out) {
+    int hb_n = H / 128, fb_n = F / 128;
+    int64_t gu_bytes = (int64_t)2 * F * H / 2, gu_sc = (int64_t)2 * F * H / 32;
+    int64_t dn_bytes = (int64_t)H * F / 2, dn_sc = (int64_t)H * F / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < T; ++t) {
+        double *xt = (double *)malloc(sizeof(double) * H);
+        double *xd = (double *)malloc(sizeof(double) * H);
+        uint8_t *xq = (uint8_t *)malloc(H);
+        float *xs = (float *)malloc(sizeof(float) * hb_n);
+        double *acc = (double *)calloc(H, sizeof(double));
+        double *wr = (double *)malloc(sizeof(double) * (H > F ? H : F));
+        double *hv = (double *)malloc(sizeof(double) * F);
+        double *hd = (double *)malloc(sizeof(double) * F);
+        uint8_t *hq = (uint8_t *)malloc(F);
+        float *hs = (float *)malloc(sizeof(float) * fb_n);
+        for (int i = 0; i < H; ++i) xt[i] = bf16_value(x[t * H + i]);
+        quantize_blocks(xt, hb_n, xq, xs);
+        for (int i = 0; i < H; ++i) xd[i] = e4m3_value(xq[i]) * (double)xs[i / 128];
+        for (int k = 0; k < K; ++k) {
+            int e = idx[t * K + k];
+            if (e < 0 || e >= E) continue;
+            contrib_mxf4(xd, w13 + e * gu_bytes, w13_sc + e * gu_sc, w2 + e * dn_bytes,
+                         w2_sc + e * dn_sc, H, F, (double)w[t * K + k], wr, hv, hd, hq, hs, acc);
+        }
+        for (int j = 0; j < H; ++j) out[t * H + j] = bf16_from_double(acc[j]);
+        free(xt); free(xd); free(xq); free(xs); free(acc); free(wr); free(hv); free(hd); free(hq);
+        free(hs);
+    }
 }
 
 #ifdef _OPENMP
