@@ -63,7 +63,9 @@ typedef enum {
 
 typedef enum {
     MOE_W_BF16 = 0,            /* bf16 expert weights, bf16 activations      */
-    MOE_W_FP8_E4M3 = 1         /* e4m3 weights with fp32 per-(row,128) scales */
+    MOE_W_FP8_E4M3 = 1,        /* e4m3 weights with fp32 per-(row,128) scales */
+    MOE_W_MXFP4 = 2            /* packed E2M1 weights, E8M0 scale per (row,32),
+                                  e4m3 activations (FP8 x FP4)                */
 } moe_wtype_t;
 
 /* Version of this ABI (incremented on any incompatible change). */
@@ -95,6 +97,17 @@ MOE_API size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe
  *   gate_up_scale  [E,2F,H/128] fp32 (e4m3 only; NULL for bf16): the value of
  *                  gate_up element (e,r,c) is e4m3(q) * gate_up_scale[e,r,c/128]
  *   down_scale     [E,H,F/128]  fp32 (e4m3 only; NULL for bf16)
+ *   MXFP4 weights (wt = MOE_W_MXFP4; "FP8 x FP4" of the GC MoE issue and the
+ *   DeepGEMM Mega MoE news page, MXFP4 of the OCP Microscaling format):
+ *     gate_up_proj [E,2F,H/2] and down_proj [E,H,F/2] bytes, two E2M1 codes
+ *                  per byte, the even column in the low nibble; 32-byte aligned
+ *     gate_up_scale / down_scale: E8M0 bytes, one per row and 32 columns,
+ *                  in the tensor cores' block layout: for each expert, one
+ *                  512-byte block per (128 rows, 128 columns) in [R/128][C/128]
+ *                  order, the scale of (r, c) at byte
+ *                  (r%32)*16 + ((r%128)/32)*4 + (c%128)/32 of its block
+ *                  (2F*H/32 and H*F/32 bytes per expert)
+ *     value of element (e,r,c) = e2m1(code) * 2^(scale - 127)
  *   out            [T,H]     bf16, fully overwritten (any device-accessible
  *                            pointer, e.g. mapped pinned host memory: the
  *                            kernels store it directly)
@@ -108,13 +121,15 @@ MOE_API size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe
  * power-of-two scale (the rule of quantize_fp8_block128), h is rounded to
  * bf16 and quantised the same way per 128 features, and each 128-long block
  * of every dot product is scaled by its activation and weight scales.
+ * MXFP4 path: the same e4m3 activations; the tensor cores apply the weight
+ * scale per 32 and the activation scale per 128 k-elements.
  * All pointers must be 16-byte aligned.
  */
 MOE_API moe_status_t moe_experts_prefill(const void *hidden_states, const void *gate_up_proj,
                                  const void *down_proj, const int32_t *top_k_index,
                                  const float *top_k_weights, int top_k, int T, int H, int F,
-                                 int E, moe_wtype_t wt, const float *gate_up_scale,
-                                 const float *down_scale, void *out, void *workspace,
+                                 int E, moe_wtype_t wt, const void *gate_up_scale,
+                                 const void *down_scale, void *out, void *workspace,
                                  size_t workspace_bytes, void *stream);
 
 /*
@@ -128,8 +143,8 @@ MOE_API moe_status_t moe_experts_prefill(const void *hidden_states, const void *
 MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_proj,
                                 const void *down_proj, const int32_t *top_k_index,
                                 const float *top_k_weights, int top_k, int T, int H, int F,
-                                int E, moe_wtype_t wt, const float *gate_up_scale,
-                                const float *down_scale, void *out, void *workspace,
+                                int E, moe_wtype_t wt, const void *gate_up_scale,
+                                const void *down_scale, void *out, void *workspace,
                                 size_t workspace_bytes, void *stream);
 
 /*
@@ -158,6 +173,7 @@ MOE_API size_t moe_experts_shared_workspace_size(int T, int H, int F, int E, int
  * precision (e4m3: the same activation quantisation and block scales).
  *
  *   arguments shared with moe_experts_prefill: same meaning and layouts
+ *   (MXFP4 routed weights return MOE_ERR_UNSUPPORTED here)
  *   shared_gate_up_proj  [S,2F,H] bf16 | e4m3 (same dtype as the routed weights)
  *   shared_down_proj     [S,H,F]  bf16 | e4m3
  *   shared_gate_up_scale [S,2F,H/128] fp32 (e4m3 only; NULL for bf16)
@@ -172,7 +188,7 @@ MOE_API size_t moe_experts_shared_workspace_size(int T, int H, int F, int E, int
 MOE_API moe_status_t moe_experts_with_shared(
     const void *hidden_states, const void *gate_up_proj, const void *down_proj,
     const int32_t *top_k_index, const float *top_k_weights, int top_k, int T, int H, int F, int E,
-    moe_wtype_t wt, const float *gate_up_scale, const float *down_scale,
+    moe_wtype_t wt, const void *gate_up_scale, const void *down_scale,
     const void *shared_gate_up_proj, const void *shared_down_proj,
     const float *shared_gate_up_scale, const float *shared_down_scale, int S,
     const void *residual, void *out, void *workspace, size_t workspace_bytes, void *stream);
@@ -191,7 +207,7 @@ MOE_API moe_status_t moe_experts_with_shared(
  * The library itself allocates nothing and calls no allocating routine.
  *  - Sizes whose decode scratch (moe_experts_workspace_size(..., 1)) exceeds
  *    1 MiB, and calls outside the decode range (T > 16 or T*K > 64), return
- *    MOE_ERR_WORKSPACE; e4m3 weights return MOE_ERR_UNSUPPORTED.
+ *    MOE_ERR_WORKSPACE; e4m3 and MXFP4 weights return MOE_ERR_UNSUPPORTED.
  *  - The first call on a device looks up the array's device address with
  *    that device current; make that first call before any stream capture.
  *  - All calls share the one array, which keeps the last call's contents:
@@ -201,8 +217,8 @@ MOE_API moe_status_t moe_experts_with_shared(
 MOE_API moe_status_t moe_experts_decode_static(const void *hidden_states, const void *gate_up_proj,
                                        const void *down_proj, const int32_t *top_k_index,
                                        const float *top_k_weights, int top_k, int T, int H, int F,
-                                       int E, moe_wtype_t wt, const float *gate_up_scale,
-                                       const float *down_scale, void *out, void *stream);
+                                       int E, moe_wtype_t wt, const void *gate_up_scale,
+                                       const void *down_scale, void *out, void *stream);
 
 /*
  * Group-aware sigmoid top-k routing (layer table:

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_W_BF16 = 0
 MOE_W_FP8_E4M3 = 1
+MOE_W_MXFP4 = 2
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 
@@ -78,12 +79,18 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _wtype(gate_up_proj):
+def _wtype(gate_up_proj, weight_format=None):
+    """bf16 -> MOE_W_BF16; float8_e4m3fn or uint8 -> MOE_W_FP8_E4M3, unless
+    weight_format == "mxfp4" (uint8 bytes of packed E2M1 codes)."""
+    if weight_format == "mxfp4":
+        if gate_up_proj.dtype != torch.uint8:
+            raise TypeError("MXFP4 weights are passed as uint8 bytes (two E2M1 codes each)")
+        return MOE_W_MXFP4
     if gate_up_proj.dtype == torch.bfloat16:
         return MOE_W_BF16
     if gate_up_proj.dtype in (torch.uint8, torch.float8_e4m3fn):
         return MOE_W_FP8_E4M3
-    raise TypeError("expert weights must be bf16 or e4m3 (uint8 / float8_e4m3fn)")
+    raise TypeError("expert weights must be bf16, e4m3 (uint8 / float8_e4m3fn) or mxfp4 bytes")
 
 
 def moe_experts_workspace_size(T, H, F, E, K, wtype=MOE_W_BF16, decode=False):
@@ -91,10 +98,14 @@ def moe_experts_workspace_size(T, H, F, E, K, wtype=MOE_W_BF16, decode=False):
 
 
 def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
-             gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None):
+             gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None,
+             weight_format=None):
     T, H = hidden_states.shape
     E, F2, H2 = gate_up_proj.shape
-    if H2 != H or down_proj.shape != (E, H, F2 // 2):
+    packed = weight_format == "mxfp4"          # two codes per byte along the reduction
+    if packed:
+        H2 *= 2
+    if H2 != H or down_proj.shape != (E, H, F2 // 2 // (2 if packed else 1)):
         raise ValueError("shape mismatch: hidden %s gate_up %s down %s" % (
             tuple(hidden_states.shape), tuple(gate_up_proj.shape), tuple(down_proj.shape)))
     if tuple(top_k_index.shape) != (T, top_k) or tuple(top_k_weights.shape) != (T, top_k):
@@ -107,7 +118,7 @@ def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_we
               down_scale):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("all tensors must be contiguous CUDA tensors")
-    wt = _wtype(gate_up_proj)
+    wt = _wtype(gate_up_proj, weight_format)
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
     decode = name == "moe_experts_decode"
@@ -123,17 +134,23 @@ def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_we
 
 
 def moe_experts_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
-                        gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None):
-    """Routed-experts forward, grouped-GEMM form.  Returns out [T,H] bf16."""
+                        gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None,
+                        weight_format=None):
+    """Routed-experts forward, grouped-GEMM form.  Returns out [T,H] bf16.
+    weight_format="mxfp4": gate_up_proj [E,2F,H/2] / down_proj [E,H,F/2] uint8
+    packed E2M1 with E8M0 scales (uint8) in the block layout."""
     return _forward("moe_experts_prefill", hidden_states, gate_up_proj, down_proj, top_k_index,
-                    top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream)
+                    top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream,
+                    weight_format)
 
 
 def moe_experts_decode(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
-                       gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None):
-    """Routed-experts forward, fused gather-GEMV form for a few tokens."""
+                       gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None,
+                       weight_format=None):
+    """Routed-experts forward, decode form for a few tokens."""
     return _forward("moe_experts_decode", hidden_states, gate_up_proj, down_proj, top_k_index,
-                    top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream)
+                    top_k_weights, top_k, gate_up_scale, down_scale, out, workspace, stream,
+                    weight_format)
 
 
 def moe_experts_shared_workspace_size(T, H, F, E, K, S, wtype=MOE_W_BF16):

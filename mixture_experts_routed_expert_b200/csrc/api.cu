@@ -35,6 +35,7 @@ struct Bump {
 };
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 moe_status_t from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return MOE_OK;
@@ -53,6 +54,13 @@ bool dims_ok(int64_t T, int H, int F, int E, int K) {
 Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t wt) {
     const int64_t N = T * K;
     const size_t eb = (wt == MOE_W_BF16) ? 2 : 1;
+    // activation scales: fp32 [N][H/128] (E4M3 weights) or E8M0 bytes in rows
+    // of round16(H/128) (MXFP4 weights); the same for h with F
+    auto scale_bytes = [&](int cols) -> size_t {
+        if (wt == MOE_W_BF16) return 0;
+        if (wt == MOE_W_MXFP4) return (size_t)N * align_up(cols / 128, 16);
+        return sizeof(float) * (size_t)N * (cols / 128);
+    };
     Workspace L;
     Bump b;
     L.status = b.take(16);
@@ -63,9 +71,9 @@ Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t w
     L.perm = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(N, 1));
     L.inv = b.take(sizeof(int32_t) * (size_t)std::max<int64_t>(N, 1));
     L.xperm = b.take(eb * (size_t)N * H);
-    L.xscale = b.take(wt == MOE_W_BF16 ? 0 : sizeof(float) * (size_t)N * (H / 128));
+    L.xscale = b.take(scale_bytes(H));
     L.h = b.take(eb * (size_t)N * F);
-    L.hscale = b.take(wt == MOE_W_BF16 ? 0 : sizeof(float) * (size_t)N * (F / 128));
+    L.hscale = b.take(scale_bytes(F));
     L.y = b.take(sizeof(float) * (size_t)N * H);
     L.total = b.off;
     return L;
@@ -108,9 +116,9 @@ bool fp8_decode_sized(int T, int K) { return T * K <= kDecodeMaxSlots; }
 
 moe_status_t check_common(const void *x, const void *gu, const void *dn, const int32_t *idx,
                           const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
-                          const float *gus, const float *dns, const void *out) {
+                          const void *gus, const void *dns, const void *out) {
     if (!dims_ok(T, H, F, E, K)) return MOE_ERR_INVALID_ARG;
-    if (wt != MOE_W_BF16 && wt != MOE_W_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+    if (wt != MOE_W_BF16 && wt != MOE_W_FP8_E4M3 && wt != MOE_W_MXFP4) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !gu || !dn || !idx || !w || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(gu) || !aligned16(dn) || !aligned16(out) ||
@@ -119,24 +127,35 @@ moe_status_t check_common(const void *x, const void *gu, const void *dn, const i
     if (wt == MOE_W_FP8_E4M3) {
         if (!gus || !dns || !aligned16(gus) || !aligned16(dns)) return MOE_ERR_INVALID_ARG;
     }
+    if (wt == MOE_W_MXFP4) {   // packed weights are read by TMA in 32-byte units
+        if (!gus || !dns || !aligned16(gus) || !aligned16(dns) || !aligned32(gu) || !aligned32(dn))
+            return MOE_ERR_INVALID_ARG;
+    }
     return MOE_OK;
 }
 
 moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const int32_t *idx,
                          const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
-                         const float *gus, const float *dns, void *out, void *ws, size_t ws_bytes,
+                         const void *gus, const void *dns, void *out, void *ws, size_t ws_bytes,
                          cudaStream_t st, int bn8 = kBNFp8, const SharedSet &sh = SharedSet(),
                          const void *residual = nullptr) {
     const Workspace L = prefill_workspace(T, H, F, E, K, wt);
     if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255)) return MOE_ERR_WORKSPACE;
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     const int64_t N = (int64_t)T * K;
-    const bool fp8 = (wt == MOE_W_FP8_E4M3);
+    const bool fp8 = (wt != MOE_W_BF16);   // E4M3 activations (E4M3 or MXFP4 weights)
     cudaError_t e = fp8 ? launch_permute_gather(x, idx, N, K, H, E, bn8, bn8, wt, wsb, L, st)
                         : launch_permute_gather(x, idx, N, K, H, E, kBNGateUp, kBNDown, wt, wsb, L, st);
-    if (e == cudaSuccess)
-        e = fp8 ? launch_gemms_fp8(gu, gus, dn, dns, w, T, H, F, E, K, bn8, wsb, L, st, sh)
-                : launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st, sh);
+    if (e == cudaSuccess) {
+        if (wt == MOE_W_MXFP4)
+            e = launch_gemms_mxf4(gu, static_cast<const uint8_t *>(gus), dn,
+                                  static_cast<const uint8_t *>(dns), w, T, H, F, E, K, bn8, wsb, L, st);
+        else if (fp8)
+            e = launch_gemms_fp8(gu, static_cast<const float *>(gus), dn,
+                                 static_cast<const float *>(dns), w, T, H, F, E, K, bn8, wsb, L, st, sh);
+        else
+            e = launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st, sh);
+    }
     if (e == cudaSuccess) e = launch_combine(idx, T, H, E, K, wsb, L, out, st, residual);
     return from_cuda(e);
 }
@@ -175,7 +194,7 @@ namespace moe {
 // Validation and decode-size rule shared with the other entry points.
 moe_status_t validate_forward(const void *x, const void *gu, const void *dn, const int32_t *idx,
                               const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
-                              const float *gus, const float *dns, const void *out) {
+                              const void *gus, const void *dns, const void *out) {
     return check_common(x, gu, dn, idx, w, K, T, H, F, E, wt, gus, dns, out);
 }
 bool decode_path_fits(int T, int K, int H, int F) { return decode_fits(T, K, H, F); }
@@ -199,7 +218,7 @@ const char *moe_status_string(moe_status_t s) {
 
 size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t wt, int decode) {
     if (!dims_ok(T, H, F, E, K)) return 0;
-    if (decode && (wt == MOE_W_BF16 || wt == MOE_W_FP8_E4M3) && decode_serves(T, K, H, F, wt))
+    if (decode && decode_serves(T, K, H, F, wt))
         return decode_workspace(T, H, F, E, K, wt).total;
     return prefill_workspace(T, H, F, E, K, wt).total;
 }
@@ -207,8 +226,8 @@ size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t
 moe_status_t moe_experts_prefill(const void *hidden_states, const void *gate_up_proj,
                                  const void *down_proj, const int32_t *top_k_index,
                                  const float *top_k_weights, int top_k, int T, int H, int F,
-                                 int E, moe_wtype_t wt, const float *gate_up_scale,
-                                 const float *down_scale, void *out, void *workspace,
+                                 int E, moe_wtype_t wt, const void *gate_up_scale,
+                                 const void *down_scale, void *out, void *workspace,
                                  size_t workspace_bytes, void *stream) {
     moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
                                   top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
@@ -222,8 +241,8 @@ moe_status_t moe_experts_prefill(const void *hidden_states, const void *gate_up_
 moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_proj,
                                 const void *down_proj, const int32_t *top_k_index,
                                 const float *top_k_weights, int top_k, int T, int H, int F, int E,
-                                moe_wtype_t wt, const float *gate_up_scale,
-                                const float *down_scale, void *out, void *workspace,
+                                moe_wtype_t wt, const void *gate_up_scale,
+                                const void *down_scale, void *out, void *workspace,
                                 size_t workspace_bytes, void *stream) {
     moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
                                   top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
@@ -234,7 +253,7 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
         return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                            top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
                            workspace_bytes, st,
-                           wt == MOE_W_FP8_E4M3 && fp8_decode_sized(T, top_k) ? kBNFp8Decode : kBNFp8);
+                           wt != MOE_W_BF16 && fp8_decode_sized(T, top_k) ? kBNFp8Decode : kBNFp8);
     const DecodeWorkspace L = decode_workspace(T, H, F, E, top_k, wt);
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
         return MOE_ERR_WORKSPACE;
@@ -252,11 +271,12 @@ size_t moe_experts_shared_workspace_size(int T, int H, int F, int E, int K, int 
 moe_status_t moe_experts_with_shared(
     const void *hidden_states, const void *gate_up_proj, const void *down_proj,
     const int32_t *top_k_index, const float *top_k_weights, int top_k, int T, int H, int F, int E,
-    moe_wtype_t wt, const float *gate_up_scale, const float *down_scale,
+    moe_wtype_t wt, const void *gate_up_scale, const void *down_scale,
     const void *shared_gate_up_proj, const void *shared_down_proj,
     const float *shared_gate_up_scale, const float *shared_down_scale, int S,
     const void *residual, void *out, void *workspace, size_t workspace_bytes, void *stream) {
     if (!shared_dims_ok(T, H, F, E, top_k, S)) return MOE_ERR_INVALID_ARG;
+    if (wt == MOE_W_MXFP4) return MOE_ERR_UNSUPPORTED;
     moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
                                   top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
                                   out);

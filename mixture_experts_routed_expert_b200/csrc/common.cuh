@@ -173,6 +173,62 @@ __device__ __forceinline__ void mma_e4m3_ss(uint32_t d_tmem, uint64_t a, uint64_
         "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// ---- block-scaled MMA (MXFP4 weights x E4M3 activations) -------------------
+// Instruction descriptor of tcgen05.mma kind::mxf8f6f4.block_scale: A = E2M1
+// (format 5), B = E4M3 (format 0), K-major A and B, E8M0 scale factors
+// (bit 23), fp32 accumulator implied, M x N tile.  The scale-factor byte
+// selectors (a_sf_id bits 29-30, b_sf_id bits 4-5) are or-ed in per MMA.
+__host__ __device__ constexpr uint32_t idesc_mxf4_e4m3(int M, int N) {
+    return (5u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_sf_ids(uint32_t a_id, uint32_t b_id) {
+    return (a_id << 29) | (b_id << 4);
+}
+// D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T with one E8M0 scale per row and 32
+// k-elements; sfa / sfb are TMEM addresses of the scale columns, their top
+// two bits selecting the byte (the 32-k slice) as in the descriptor.
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+// Shared-memory descriptor of a 32-row x 16-byte block without swizzle (rows
+// 16 bytes apart, 8-row groups 128 bytes apart): the source of
+// tcgen05.cp 32x128b.
+__device__ __forceinline__ uint64_t sdesc_rows16(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);        // start address
+    d |= (uint64_t)(128 >> 4) << 32;                // stride byte offset: next 8 rows
+    d |= (uint64_t)1 << 46;                         // descriptor version
+    return d;                                       // layout type 0: no swizzle
+}
+// Copy 32 rows x 128 bits from shared memory into TMEM columns [taddr,
+// taddr+4) of all four 32-lane quarters (row i -> lane i of every quarter).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+// Non-tensor bulk copy global -> shared (16-byte aligned, bytes % 16 == 0),
+// completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                          uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to later
+// async-proxy reads (TMA, tcgen05.cp, tcgen05.mma).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Arrive once on `bar` when every MMA issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile(

@@ -1,0 +1,468 @@
+// gemm_mxf4.cu -- S4 and S5 of the prefill path for MXFP4 routed weights
+// (packed E2M1, one E8M0 scale per row and 32 columns) with E4M3 activations
+// (power-of-two scale per 128 columns): the FP8 x FP4 precision of the GC MoE
+// issue ("FP8 activations, packed FP4 routed weights") and of DeepGEMM's Mega
+// MoE (news page: "FP8 x FP4"; sgl-deep-gemm commit list: "MXF4 kind").
+//
+// Grouped GEMM on tcgen05 with kind::mxf8f6f4.block_scale: the tensor cores
+// apply both scales (per 32 k-elements) themselves, so every tile accumulates
+// its whole K range in TMEM with no per-k-block promotion.
+//   - weights: TMA with the 16U4_ALIGN16B type expands every 16 packed E2M1
+//     codes (8 bytes) into a 16-byte slot, giving the same 128-byte rows per
+//     128 k-elements as E4M3 and the same 128-byte-swizzled operand tiles;
+//   - weight scales are stored in the tensor cores' block layout (a 512-byte
+//     block per 128 rows x 128 columns) and arrive with one bulk copy per
+//     k-block and operand;
+//   - activation scales: the producer warp expands each routed row's E8M0
+//     byte (the power-of-two block-128 scale) into the same block layout in
+//     shared memory (the byte repeated for the four 32-element slices);
+//   - the MMA warp copies the scale blocks into TMEM (tcgen05.cp 32x128b,
+//     all four lane quarters) and issues four MMAs of K = 32 per k-block,
+//     each selecting its scale byte.
+// Tiles, warp roles and epilogues as in the E4M3 kernel: warp 0 TMA producer,
+// warp 1 TMEM allocation + MMA issue, warps 2-9 epilogue from double-buffered
+// TMEM accumulators.
+//   S4 (gate_up): h = bf16(SiLU(g) * u), quantised per 128 features (the
+//     tile's rows) to E4M3 with a power-of-two scale -> hq [N][F] and the
+//     scale's E8M0 byte -> hsf [N][FBp].
+//   S5 (down): y[slot, j] = w[slot] * acc (fp32, by original slot).
+#include "common.cuh"
+#include "gemm_common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kEpiF = 8;
+constexpr int kThreadsF = 64 + 32 * kEpiF;
+constexpr int kMaxKBF = 128;          // k-blocks (of 128) per row supported
+
+template <bool GATE_UP, int BN>
+struct CfgF {
+    static_assert(BN == 64 || BN == 16, "one epilogue thread owns 32 or 8 columns");
+    static constexpr int NUM_A = GATE_UP ? 2 : 1;
+    static constexpr int MAX_STAGES = 12;
+    static constexpr int BOX = BN < 32 ? BN : 32;       // routed rows per TMA box
+    static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 E2M1 in 16-byte slots
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int SF_OFF = NUM_A * A_BYTES + B_BYTES;   // scale blocks: [A0][A1][B]
+    static constexpr int STAGE_BYTES = (SF_OFF + (NUM_A + 1) * 512 + 1023) / 1024 * 1024;
+    static constexpr int ACC = NUM_A * BN;              // TMEM columns of one accumulator set
+    static constexpr int SF_COL = 2 * ACC;              // scale columns after the two sets
+    static constexpr int COLS_USED = SF_COL + 4 * (NUM_A + 1);
+    static constexpr int TMEM_COLS =
+        COLS_USED <= 64 ? 64 : (COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512));
+    static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
+    static constexpr int NC = BN / 2;                   // columns per epilogue thread
+    static size_t smem_bytes(int E, int KBp, int stages) {
+        return 1024 + (size_t)stages * STAGE_BYTES + 1024 + (size_t)BN * KBp +
+               sizeof(float) * 5 * BN + 2 * sizeof(int) * (E + 1) + 64;
+    }
+};
+
+struct GemmFArgs {
+    const int32_t *offsets, *tiles;
+    int E, MT, KB;
+    int a_rows_per_expert, up_offset;
+    const uint8_t *wsf;          // E8M0 weight scales in the block layout
+    int64_t wsf_per_expert;      // bytes of one expert's weight scales
+    const uint8_t *xsf;          // [N][KBp] E8M0 activation scales of the routed rows
+    int KBp;                     // row stride of xsf (k-blocks rounded up to 16)
+    uint8_t *hq;                 // gate_up: [N][F] e4m3
+    uint8_t *hsf;                // gate_up: [N][FBp] E8M0
+    int F, FBp;
+    float *y;                    // down: [T*K][H]
+    int H;
+    const int32_t *perm;
+    const float *topw;
+    int32_t *status;
+    int stages;                  // depth of the TMA ring (2..MAX_STAGES)
+};
+
+__device__ __forceinline__ void epi_sync_f() {
+    asm volatile("bar.sync 2, %0;" ::"n"(32 * kEpiF) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+
+template <bool GATE_UP, int BN>
+__global__ void __launch_bounds__(kThreadsF, 1)
+    grouped_gemm_mxf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const GemmFArgs args) {
+    using C = CfgF<GATE_UP, BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ring = smem;
+    const int NST = args.stages;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)NST * C::STAGE_BYTES);
+    uint64_t *empty = full + C::MAX_STAGES;
+    uint64_t *afull = empty + C::MAX_STAGES;
+    uint64_t *aempty = afull + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(aempty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    uint8_t *sxs = smem + (size_t)NST * C::STAGE_BYTES + 1024;           // [BN][KBp]
+    float *amax_s = reinterpret_cast<float *>(sxs + (size_t)BN * args.KBp);   // [4][BN]
+    float *scale_s = amax_s + 4 * BN;                                    // [BN]
+    int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + BN);
+    int32_t *s_tiles = s_off + (args.E + 1);
+    const int KB = args.KB;
+
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afull[b], 1);
+            mbar_init(&aempty[b], 32 * kEpiF);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    pdl_wait();
+    for (int i = threadIdx.x; i <= args.E; i += blockDim.x) {
+        s_off[i] = args.offsets[i];
+        s_tiles[i] = args.tiles[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = s_tiles[args.E] * args.MT;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        const uint64_t pol_once = policy_evict_first();
+        const uint64_t pol_x = policy_evict_last();
+        const int KBp = args.KBp;
+        int stage = 0, armed[C::MAX_STAGES];
+        uint32_t phase = 0;
+        for (int s = 0; s < C::MAX_STAGES; ++s) armed[s] = -1;
+        bool ok = true;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+            const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
+            // the tile's activation-scale bytes, row n -> sxs[n][0..KBp)
+            const int nch = KBp / 16;
+            for (int i = lane; i < t.nrows * nch; i += 32) {
+                const int n = i / nch, c = i - n * nch;
+                cp_async16(sxs + n * KBp + 16 * c, args.xsf + (size_t)(t.row0 + n) * KBp + 16 * c);
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncwarp();
+            const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
+            const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
+            const uint32_t bytes = C::NUM_A * (C::A_BYTES + 512) + nbox * C::BOX * 128;
+            const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
+            const uint8_t *sfa0 = args.wsf + t.e * args.wsf_per_expert + (size_t)t.m * KB * 512;
+            const uint8_t *sfa1 = sfa0 + (size_t)(args.up_offset / kBM) * KB * 512;
+            for (int kb = 0; kb < KB; ++kb) {
+                if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                uint8_t *sA = ring + stage * C::STAGE_BYTES;
+                uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
+                uint8_t *sF = sA + C::SF_OFF;
+                uint32_t *sfb = reinterpret_cast<uint32_t *>(sF + C::NUM_A * 512);
+                // activation scales in the block layout: column n at word
+                // (n % 32) * 4 + n / 32, its byte repeated for the 4 slices
+                for (int n = lane; n < BN; n += 32) {
+                    const uint32_t b = n < t.nrows ? (uint32_t)sxs[n * KBp + kb] : 127u;
+                    sfb[(n & 31) * 4 + (n >> 5)] = b * 0x01010101u;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    armed[stage] = (int)phase;
+                    tma_load_2d(sA, &tmA, &full[stage], kb * 128, arow, pol_w);
+                    bulk_load(sF, sfa0 + (size_t)kb * 512, 512, &full[stage], pol_w);
+                    if (GATE_UP) {
+                        tma_load_2d(sA + C::A_BYTES, &tmA, &full[stage], kb * 128,
+                                    arow + args.up_offset, pol_w);
+                        bulk_load(sF + 512, sfa1 + (size_t)kb * 512, 512, &full[stage], pol_w);
+                    }
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(sB + b * C::BOX * 128, &tmB, &full[stage], kb * 128,
+                                    t.row0 + b * C::BOX, pol_x);
+                }
+                if (++stage == NST) { stage = 0; phase ^= 1; }
+            }
+        }
+        if (lane == 0) {
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+            }
+            volatile int never = 0;
+            for (int s = 0; s < NST; ++s)
+                if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
+                    atomicOr(args.status, DEV_TIMEOUT);
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------- MMA issue ----
+        if (lane == 0) {
+            int stage = 0, ab = 0;
+            uint32_t phase = 0, aphase = 0;
+            bool ok = true;
+            const uint32_t tsf = tmem_base + C::SF_COL;       // A0 scales; A1 at +4; B at +4*NUM_A
+            const uint32_t tsfb = tsf + 4 * C::NUM_A;
+            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
+                const uint32_t idesc = idesc_mxf4_e4m3(kBM, (t.nrows + 15) & ~15);
+                if (!mbar_wait(&aempty[ab], aphase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem_base + ab * C::ACC;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(ring + stage * C::STAGE_BYTES);
+                    const uint32_t sf = sa + C::SF_OFF;
+                    tmem_cp_32x128b_x4(tsf, sdesc_rows16(sf));
+                    if (GATE_UP) tmem_cp_32x128b_x4(tsf + 4, sdesc_rows16(sf + 512));
+                    tmem_cp_32x128b_x4(tsfb, sdesc_rows16(sf + C::NUM_A * 512));
+                    const uint64_t da = sdesc_sw128(sa);
+                    const uint64_t da2 = sdesc_sw128(sa + C::A_BYTES);
+                    const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t id = idesc | idesc_sf_ids(k, k);
+                        const uint32_t sel = (uint32_t)k << 30;
+                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                        mma_mxf4_ss(d, da + 2 * k, db + 2 * k, id, tsf | sel, tsfb | sel, acc);
+                        if (GATE_UP)
+                            mma_mxf4_ss(d + BN, da2 + 2 * k, db + 2 * k, id, (tsf + 4) | sel,
+                                        tsfb | sel, acc);
+                    }
+                    mma_commit(&empty[stage]);
+                    if (++stage == NST) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&afull[ab]);
+                if (++ab == 2) { ab = 0; aphase ^= 1; }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- epilogue ----
+        constexpr int NC = C::NC;
+        const int ew = warp - 2, et = threadIdx.x - 64;
+        const int eg = warp & 3;                 // TMEM lanes [32*eg, 32*eg+32)
+        const int half = ew >> 2;                // columns [NC*half, NC*half+NC)
+        const int row = eg * 32 + lane;
+        int ab = 0;
+        uint32_t aphase = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < total; w += gridDim.x) {
+            const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
+            const int live = t.nrows - half * NC;   // columns of this thread that hold routed rows
+            if (ok && !mbar_wait(&afull[ab], aphase, abort_flag)) {
+                ok = false;
+                *abort_flag = 1;
+                atomicOr(args.status, DEV_TIMEOUT);
+            }
+            tc_fence_after();
+            const uint32_t ta = tmem_base + ((uint32_t)(eg * 32) << 16) + ab * C::ACC + half * NC;
+            float ag[NC], au[GATE_UP ? NC : 1];
+            {
+                uint32_t r[NC];
+                if constexpr (NC == 32) tmem_ld32(ta, r); else tmem_ld8(ta, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < NC; ++j) ag[j] = __uint_as_float(r[j]);
+                if (GATE_UP) {
+                    if constexpr (NC == 32) tmem_ld32(ta + BN, r); else tmem_ld8(ta + BN, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < NC; ++j) au[j] = __uint_as_float(r[j]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&aempty[ab]);
+            if (++ab == 2) { ab = 0; aphase ^= 1; }
+            if (GATE_UP) {
+                // h = bf16(SiLU(g) * u) for this row (feature) and NC routed rows
+#pragma unroll
+                for (int j = 0; j < NC; ++j)
+                    ag[j] = __bfloat162float(__float2bfloat16_rn(silu_f(ag[j]) * au[j]));
+                // column max of |h| over this warp's 32 rows: lane l ends
+                // with column l of each group of 32
+#pragma unroll
+                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = 32 * grp + j < NC ? fabsf(ag[32 * grp + j]) : 0.f;
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+                        for (int i = 0; i < o; ++i) {
+                            const bool upper = (lane & o) != 0;
+                            const float send = upper ? v[i] : v[i + o];
+                            const float keep = upper ? v[i + o] : v[i];
+                            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
+                        }
+                    }
+                    if (32 * grp + lane < NC) amax_s[eg * BN + half * NC + 32 * grp + lane] = v[0];
+                }
+                epi_sync_f();
+                if (et < BN) {
+                    const float m = fmaxf(fmaxf(amax_s[et], amax_s[BN + et]),
+                                          fmaxf(amax_s[2 * BN + et], amax_s[3 * BN + et]));
+                    const int k = fp8_block_exp(m);
+                    scale_s[et] = pow2f(-k);
+                    if (et < t.nrows)
+                        args.hsf[(size_t)(t.row0 + et) * args.FBp + t.m] = (uint8_t)(k + 127);
+                }
+                epi_sync_f();
+                uint8_t *hp = args.hq + (size_t)(t.row0 + half * NC) * args.F + t.m * kBM + row;
+#pragma unroll
+                for (int j = 0; j < NC; ++j) {
+                    if (j < live)
+                        hp[(size_t)j * args.F] =
+                            (uint8_t)(e4m3x2(ag[j] * scale_s[half * NC + j], 0.f) & 0xFF);
+                }
+                epi_sync_f();                    // scale_s is rewritten by the next tile
+            } else {
+                float *yp = args.y + t.m * kBM + row;
+#pragma unroll
+                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
+                    const int c = half * NC + 32 * grp + lane;
+                    const int my_slot = (c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
+                    const float my_w = (c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                        const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                        if (32 * grp + j < NC && 32 * grp + j < live)
+                            yp[(size_t)slot * args.H] = wj * ag[32 * grp + j];
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+template <bool GATE_UP, int BN>
+cudaError_t launch_oneF(const CUtensorMap &a, const CUtensorMap &b, const GemmFArgs &args,
+                        cudaStream_t st) {
+    using C = CfgF<GATE_UP, BN>;
+    static size_t attr_bytes[64] = {};          // per device: dynamic shared memory limit set so far
+    int dev = 0;
+    cudaGetDevice(&dev);
+    constexpr size_t kSmemMax = 227 * 1024;
+    GemmFArgs af = args;
+    af.stages = C::MAX_STAGES;
+    while (af.stages > 2 && C::smem_bytes(args.E, args.KBp, af.stages) > kSmemMax) --af.stages;
+    const size_t need = C::smem_bytes(args.E, args.KBp, af.stages);
+    if (need > kSmemMax) return cudaErrorInvalidValue;
+    if (attr_bytes[dev & 63] < need) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_mxf4<GATE_UP, BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need);
+        if (e != cudaSuccess) return e;
+        attr_bytes[dev & 63] = need;
+    }
+    return launch_k(grouped_gemm_mxf4<GATE_UP, BN>, dim3(num_sms()), dim3(kThreadsF), need, st, true,
+                    a, b, af);
+}
+
+// Packed E2M1 matrix [rows][cols] (cols/2 bytes a row): boxes of 128 rows x
+// 128 elements, each 16 codes expanded to a 16-byte slot in shared memory,
+// 128-byte swizzle.
+bool make_tmap_e2m1(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols / 2};
+    cuuint32_t box[2] = {128, (cuuint32_t)kBM};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(ptr), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_gemms_mxf4(const void *w13, const uint8_t *w13sf, const void *w2,
+                              const uint8_t *w2sf, const float *topw, int64_t T, int H, int F,
+                              int E, int K, int bn, uint8_t *ws, const Workspace &L,
+                              cudaStream_t st) {
+    if (H / 128 > kMaxKBF || F / 128 > kMaxKBF) return cudaErrorInvalidValue;
+    if (bn != kBNFp8 && bn != kBNFp8Decode) return cudaErrorInvalidValue;
+    const int box = bn < 32 ? bn : 32;
+    const uint64_t N = (uint64_t)T * K;
+    CUtensorMap ta, tb, tc, td;
+    const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    if (!make_tmap_e2m1(&ta, w13, (uint64_t)E * 2 * F, H) ||
+        !make_tmap(&tb, U8, 1, ws + L.xperm, N, H, box) ||
+        !make_tmap_e2m1(&tc, w2, (uint64_t)E * H, F) ||
+        !make_tmap(&td, U8, 1, ws + L.h, N, F, box))
+        return cudaErrorInvalidValue;
+    GemmFArgs g = {};
+    g.offsets = (const int32_t *)(ws + L.offsets);
+    g.E = E;
+    g.perm = (const int32_t *)(ws + L.perm);
+    g.topw = topw;
+    g.status = (int32_t *)(ws + L.status);
+    g.hq = ws + L.h;
+    g.hsf = ws + L.hscale;
+    g.F = F;
+    g.FBp = (int)align_up(F / 128, 16);
+    g.y = (float *)(ws + L.y);
+    g.H = H;
+
+    GemmFArgs a1 = g;
+    a1.tiles = (const int32_t *)(ws + L.tiles_g);
+    a1.MT = F / kBM;
+    a1.KB = H / 128;
+    a1.a_rows_per_expert = 2 * F;
+    a1.up_offset = F;
+    a1.wsf = w13sf;
+    a1.wsf_per_expert = (int64_t)2 * F * H / 32;
+    a1.xsf = ws + L.xscale;
+    a1.KBp = (int)align_up(H / 128, 16);
+
+    GemmFArgs a2 = g;
+    a2.tiles = (const int32_t *)(ws + L.tiles_d);
+    a2.MT = H / kBM;
+    a2.KB = F / 128;
+    a2.a_rows_per_expert = H;
+    a2.up_offset = 0;
+    a2.wsf = w2sf;
+    a2.wsf_per_expert = (int64_t)H * F / 32;
+    a2.xsf = ws + L.hscale;
+    a2.KBp = g.FBp;
+    if (bn == kBNFp8Decode) {
+        const cudaError_t err = launch_oneF<true, kBNFp8Decode>(ta, tb, a1, st);
+        if (err != cudaSuccess) return err;
+        return launch_oneF<false, kBNFp8Decode>(tc, td, a2, st);
+    }
+    const cudaError_t err = launch_oneF<true, kBNFp8>(ta, tb, a1, st);
+    if (err != cudaSuccess) return err;
+    return launch_oneF<false, kBNFp8>(tc, td, a2, st);
+}
+
+}  // namespace moe

@@ -51,7 +51,7 @@ constexpr int kDecodeMaxT = 16;
 // Host-side argument checks of the forward entry points (MOE_OK when valid).
 moe_status_t validate_forward(const void *x, const void *gu, const void *dn, const int32_t *idx,
                               const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
-                              const float *gus, const float *dns, const void *out);
+                              const void *gus, const void *dns, const void *out);
 // True when T tokens x K slots are served by the decode kernels.
 bool decode_path_fits(int T, int K, int H, int F);
 
@@ -86,6 +86,12 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
                              uint8_t *ws, const Workspace &L, cudaStream_t st,
                              const SharedSet &sh = SharedSet());
 // residual: optional [T][H] bf16 added after the slot sum (nullptr: none).
+// MXFP4 weights (packed E2M1 + E8M0 scales in the block layout), E4M3
+// activations with E8M0 scale bytes in the workspace's scale regions.
+cudaError_t launch_gemms_mxf4(const void *w13, const uint8_t *w13sf, const void *w2,
+                              const uint8_t *w2sf, const float *topw, int64_t T, int H, int F,
+                              int E, int K, int bn, uint8_t *ws, const Workspace &L,
+                              cudaStream_t st);
 cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, const uint8_t *ws,
                            const Workspace &L, void *out, cudaStream_t st,
                            const void *residual = nullptr);

@@ -67,7 +67,8 @@ __device__ int block_scan_inplace(int32_t *v, int n) {
 }
 
 // MODE 0: permutation only; 1: + bf16 row gather; 2: + gather with block-128
-// E4M3 quantisation (the rule of quantize_fp8_block128).
+// E4M3 quantisation (the rule of quantize_fp8_block128), fp32 scales [N][H/128];
+// 3: as 2, scales stored as E8M0 bytes in rows of round16(H/128) bytes.
 // Block (b, c) handles slots [b*chunk, (b+1)*chunk), chunk <= kPThreads, and
 // gathers column slice c of their rows (gridDim.y slices of whole 128-column
 // blocks, so that a few slots still spread over many blocks); only blocks
@@ -194,7 +195,15 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
                 const uint2 q = quant8_e4m3(f, sc);   // every lane takes part
                 if (on) {
                     dst[v] = q;
-                    if ((lane & 15) == 0) xscale[(size_t)p * (H / 128) + v / 16] = sc;
+                    if ((lane & 15) == 0) {
+                        if (MODE == 2) {
+                            xscale[(size_t)p * (H / 128) + v / 16] = sc;
+                        } else {   // E8M0 byte of the power-of-two scale, rows of KBp bytes
+                            const int kbp = (H / 128 + 15) & ~15;
+                            reinterpret_cast<uint8_t *>(xscale)[(size_t)p * kbp + v / 16] =
+                                (uint8_t)((__float_as_uint(sc) >> 23) & 0xFF);
+                        }
+                    }
                 }
             }
         }
@@ -317,6 +326,7 @@ cudaError_t launch_permute_gather(const void *x, const int32_t *idx, int64_t n_s
                                   int E, int bn_g, int bn_d, moe_wtype_t wt, uint8_t *ws,
                                   const Workspace &L, cudaStream_t st) {
     if (wt == MOE_W_BF16) return launch_pg<1>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
+    if (wt == MOE_W_MXFP4) return launch_pg<3>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
     return launch_pg<2>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
 }
 

@@ -59,7 +59,7 @@ using namespace moe;
 extern "C" MOE_API moe_status_t moe_experts_decode_static(
     const void *hidden_states, const void *gate_up_proj, const void *down_proj,
     const int32_t *top_k_index, const float *top_k_weights, int top_k, int T, int H, int F, int E,
-    moe_wtype_t wt, const float *gate_up_scale, const float *down_scale, void *out,
+    moe_wtype_t wt, const void *gate_up_scale, const void *down_scale, void *out,
     void *stream) {
     moe_status_t s = validate_forward(hidden_states, gate_up_proj, down_proj, top_k_index,
                                       top_k_weights, top_k, T, H, F, E, wt, gate_up_scale,

@@ -94,3 +94,24 @@ def test_shared_entry_host_checks(mod):
     assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 1, p, p, p, p, N, N, 2, N, p, p, big, N) == 1
     # workspace too small
     assert f(p, p, p, p, p, 6, 4, 1280, 896, 64, 0, N, N, p, p, N, N, 2, N, p, p, 4096, N) == 3
+
+
+def test_mxfp4_host_checks(mod):
+    """MXFP4 weights: scales required, weights 32-byte aligned; workspace
+    holds E8M0 scale bytes; no shared-expert or static-scratch form."""
+    L = mod.lib
+    N = None
+    p = ctypes.c_void_p(0x1000)
+    p16 = ctypes.c_void_p(0x1010)            # 16- but not 32-byte aligned
+    big = 1 << 34
+    W = mod.MOE_W_MXFP4
+    assert W == 2
+    assert L.moe_experts_prefill(p, p, p, p, p, 8, 4, 7168, 2048, 256, W, N, N, p, p, big, N) == 1
+    assert L.moe_experts_prefill(p, p16, p, p, p, 8, 4, 7168, 2048, 256, W, p, p, p, p, big, N) == 1
+    assert L.moe_experts_prefill(p, p, p, p, p, 8, 4, 7168, 2048, 256, W, p, p, p, p, 64, N) == 3
+    ws = mod.moe_experts_workspace_size
+    assert 0 < ws(64, 7168, 2048, 256, 8, W) < ws(64, 7168, 2048, 256, 8, mod.MOE_W_FP8_E4M3)
+    assert ws(4, 7168, 2048, 256, 8, W, decode=True) == ws(4, 7168, 2048, 256, 8, W)
+    f = L.moe_experts_with_shared
+    assert f(p, p, p, p, p, 8, 4, 7168, 2048, 256, W, p, p, p, p, N, N, 1, N, p, p, big, N) == 2
+    assert L.moe_experts_decode_static(p, p, p, p, p, 6, 1, 1280, 896, 64, W, p, p, p, N) == 2
