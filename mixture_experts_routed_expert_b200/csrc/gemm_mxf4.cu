@@ -167,7 +167,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             __syncwarp();
             const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
             const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
-            const uint32_t bytes = C::NUM_A * (C::A_BYTES + 512) + nbox * C::BOX * 128;
+            // the E2M1 loads count their packed bytes (half the 16-byte slots)
+            const uint32_t bytes = C::NUM_A * (C::A_BYTES / 2 + 512) + nbox * C::BOX * 128;
             const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
             const uint8_t *sfa0 = args.wsf + t.e * args.wsf_per_expert + (size_t)t.m * KB * 512;
             const uint8_t *sfa1 = sfa0 + (size_t)(args.up_offset / kBM) * KB * 512;
