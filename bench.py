@@ -479,9 +479,50 @@ def run_ours(args):
         breakdown["fp8_dsv3_shared1_residual_T%d" % T] = dict(
             fp8_entry(T, None, args.steps, S=1), entry="with_shared",
             includes="router + quantise + routed and shared experts + residual")
+    # the same layer with MXFP4 routed weights (FP8 activations x FP4 weights)
+    del fp8_w
+    mx_w = inputs.mxf4_weights(seed=0, device=dev)
+    per_expert_mxf4 = 3 * D["F"] * D["H"] // 2 + 3 * D["F"] * D["H"] // 32
+
+    def mxf4_entry(T, zipf, steps):
+        lay = inputs.fp8_layer(T, seed=T, device=dev, weights=(None, None, None, None), zipf=zipf)
+        idx = torch.empty(T, D["K"], dtype=torch.int32, device=dev)
+        tw = torch.empty(T, D["K"], dtype=torch.float32, device=dev)
+        out = torch.empty(T, D["H"], dtype=torch.bfloat16, device=dev)
+        dec = T * D["K"] <= 64
+        wsz = moe.moe_experts_workspace_size(T, D["H"], D["F"], D["E"], D["K"], moe.MOE_W_MXFP4, dec)
+        ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
+        fn = moe.moe_experts_decode if dec else moe.moe_experts_prefill
+
+        def call():
+            moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"], D["topk_group"],
+                                          D["K"], D["scale"], top_k_index=idx, top_k_weights=tw)
+            fn(lay.x, mx_w[0], mx_w[2], idx, tw, D["K"], gate_up_scale=mx_w[1],
+               down_scale=mx_w[3], out=out, workspace=ws, weight_format="mxfp4")
+        t, g = time_graph(call, steps, args.warmup)
+        us = float(np.mean(t))
+        n_t = len(set(idx.cpu().reshape(-1).tolist()))
+        byts = n_t * per_expert_mxf4 + T * D["H"] * 4 + T * D["E"] * 4
+        flops = 6 * T * D["K"] * D["H"] * D["F"]
+        t_hbm = byts / (peaks["hbm"] * 1e3)
+        t_tc = flops / (2 * peaks["bf16"] * 1e6)
+        del g
+        return dict(us=round(us, 2), touched_experts=n_t, gbs=round(byts / us / 1e3, 1),
+                    tflops=round(flops / us / 1e6, 1), hbm_frac=round(t_hbm / us, 3),
+                    tc_frac=round(t_tc / us, 3), roofline_frac=round(max(t_hbm, t_tc) / us, 3),
+                    bound="hbm" if t_hbm > t_tc else "tensor",
+                    entry="decode" if dec else "prefill",
+                    includes="router + quantise + experts (MXFP4 weights)")
+
+    for T in (128, 8, 1):
+        breakdown["mxf4_dsv3_T%d" % T] = mxf4_entry(T, None, args.steps)
     # skewed sweep (Zipf 1.1 expert popularity), FP8 and the OCR-2 bf16 shape
     sweep_steps = max(3, min(args.steps, 10))
     sweep = {}
+    for T in (1, 8, 64, 512, 2048, 8192):
+        sweep["mxf4_T%d" % T] = mxf4_entry(T, 1.1, sweep_steps)
+    del mx_w
+    fp8_w = inputs.fp8_weights(seed=0, device=dev)
     for T in (1, 8, 64, 512, 2048, 8192):
         sweep["fp8_T%d" % T] = fp8_entry(T, 1.1, sweep_steps)
     del fp8_w
@@ -587,6 +628,25 @@ def run_only(args):
         torch.cuda.synchronize()
         print("ok", args.only, float(out.float().abs().sum()))
         return
+    if args.only in ("mxf4_small", "mxf4_dec_small", "mxf4_big"):
+        # the DeepSeek-V3 expert shapes with MXFP4 weights and 32 experts
+        # (0.75 GB): T=16 prefill, T=1 decode, T=2048 prefill
+        D = dict(inputs.DSV3_FP8)
+        D["E"] = 32
+        T = {"mxf4_small": 16, "mxf4_dec_small": 1, "mxf4_big": 2048}[args.only]
+        fwd = moe.moe_experts_decode if args.only == "mxf4_dec_small" else moe.moe_experts_prefill
+        w13, w13s, w2, w2s = inputs.mxf4_weights(seed=0, device=dev, E=D["E"])
+        lay = inputs.fp8_layer(T, seed=T, device=dev, E=D["E"], weights=(None, None, None, None))
+        flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        for i in range(args.warmup + args.steps):
+            flush_w.fill_(i & 0xFF)
+            idx, tw = moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"],
+                                                    D["topk_group"], D["K"], D["scale"])
+            out = fwd(lay.x, w13, w2, idx, tw, D["K"], gate_up_scale=w13s, down_scale=w2s,
+                      weight_format="mxfp4")
+        torch.cuda.synchronize()
+        print("ok", args.only, float(out.float().abs().sum()))
+        return
     T = {"decode1": 1, "decode4": 4, "prefill2048": 2048}[args.only]
     fn = moe.moe_experts_prefill if args.only.startswith("prefill") else moe.moe_experts_decode
     lay = inputs.ocr2_layer(T, seed=T, device=dev)
@@ -671,7 +731,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048", "fp8_128", "fp8_small",
-                                       "fp8_dec_small", "fp8_big"],
+                                       "fp8_dec_small", "fp8_big", "mxf4_small", "mxf4_dec_small",
+                                       "mxf4_big"],
                     default=None,
                     help="run just W+K eager calls of one workload (for profiler captures)")
     args = ap.parse_args()
