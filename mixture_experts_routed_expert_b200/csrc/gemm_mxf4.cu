@@ -19,9 +19,12 @@
 //   - the MMA warp copies the scale blocks into TMEM (tcgen05.cp 32x128b,
 //     all four lane quarters) and issues four MMAs of K = 32 per k-block,
 //     each selecting its scale byte.
-// Tiles, warp roles and epilogues as in the E4M3 kernel: warp 0 TMA producer,
-// warp 1 TMEM allocation + MMA issue, warps 2-9 epilogue from double-buffered
-// TMEM accumulators.
+// Tiles and epilogues as in the E4M3 kernel.  Warp roles: warp 0 TMA
+// producer, warp 1 TMEM allocation + MMA issue for the gate (or down) operand,
+// warps 2-9 epilogue from double-buffered TMEM accumulators, warp 10 (gate_up
+// only) MMA issue for the up operand: with a few routed rows per tile an MMA
+// instruction does little tensor work, and two issuing warps keep the tensor
+// cores fed where one could not.
 //   S4 (gate_up): h = bf16(SiLU(g) * u), quantised per 128 features (the
 //     tile's rows) to E4M3 with a power-of-two scale -> hq [N][F] and the
 //     scale's E8M0 byte -> hsf [N][FBp].
@@ -35,22 +38,28 @@ namespace moe {
 namespace {
 
 constexpr int kEpiF = 8;
-constexpr int kThreadsF = 64 + 32 * kEpiF;
 constexpr int kMaxKBF = 128;          // k-blocks (of 128) per row supported
 
 template <bool GATE_UP, int BN>
 struct CfgF {
     static_assert(BN == 64 || BN == 16, "one epilogue thread owns 32 or 8 columns");
     static constexpr int NUM_A = GATE_UP ? 2 : 1;
+    // one MMA-issuing warp per A operand (gate, up): the issue of block-scaled
+    // MMAs with few routed rows, not the tensor cores, paces a k-block
+    static constexpr int THREADS = 64 + 32 * kEpiF + 32 * (NUM_A - 1);
     static constexpr int MAX_STAGES = 12;
-    static constexpr int BOX = BN < 32 ? BN : 32;       // routed rows per TMA box
-    static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 E2M1 in 16-byte slots
-    static constexpr int B_BYTES = BN * 128;
-    static constexpr int SF_OFF = NUM_A * A_BYTES + B_BYTES;   // scale blocks: [A0][A1][B]
-    static constexpr int STAGE_BYTES = (SF_OFF + (NUM_A + 1) * 512 + 1023) / 1024 * 1024;
+    // k-blocks per pipeline stage: one 3-D TMA load per operand and stage, so
+    // that the producer's issue cost per byte halves
+    static constexpr int KPB = 2;
+    static constexpr int A_KB = kBM * 128;              // 128 rows x 128 E2M1 in 16-byte slots
+    static constexpr int A_BYTES = KPB * A_KB;          // one operand, one stage: [kb][row][128]
+    static constexpr int B_KB = BN * 128;
+    static constexpr int B_BYTES = KPB * B_KB;          // [kb][routed row][128]
+    static constexpr int SF_OFF = NUM_A * A_BYTES + B_BYTES;   // scale blocks: [A0][A1][B] x KPB
+    static constexpr int STAGE_BYTES = (SF_OFF + (NUM_A + 1) * KPB * 512 + 1023) / 1024 * 1024;
     static constexpr int ACC = NUM_A * BN;              // TMEM columns of one accumulator set
     static constexpr int SF_COL = 2 * ACC;              // scale columns after the two sets
-    static constexpr int COLS_USED = SF_COL + 4 * (NUM_A + 1);
+    static constexpr int COLS_USED = SF_COL + 8 * NUM_A;   // per operand: A and B scale columns
     static constexpr int TMEM_COLS =
         COLS_USED <= 64 ? 64 : (COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512));
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
@@ -90,7 +99,7 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
 }
 
 template <bool GATE_UP, int BN>
-__global__ void __launch_bounds__(kThreadsF, 1)
+__global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
     grouped_gemm_mxf4(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const GemmFArgs args) {
     using C = CfgF<GATE_UP, BN>;
@@ -116,10 +125,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], C::NUM_A);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&afull[b], 1);
+            mbar_init(&afull[b], C::NUM_A);
             mbar_init(&aempty[b], 32 * kEpiF);
         }
         *abort_flag = 0;
@@ -166,41 +175,44 @@ __global__ void __launch_bounds__(kThreadsF, 1)
             cp_async_wait<0>();
             __syncwarp();
             const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
-            const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
-            // the E2M1 loads count their packed bytes (half the 16-byte slots)
-            const uint32_t bytes = C::NUM_A * (C::A_BYTES / 2 + 512) + nbox * C::BOX * 128;
             const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
             const uint8_t *sfa0 = args.wsf + t.e * args.wsf_per_expert + (size_t)t.m * KB * 512;
             const uint8_t *sfa1 = sfa0 + (size_t)(args.up_offset / kBM) * KB * 512;
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb0 = 0; kb0 < KB; kb0 += C::KPB) {
+                const int nkb = min(C::KPB, KB - kb0);
                 if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag);
                 ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
                 if (!ok) break;
                 uint8_t *sA = ring + stage * C::STAGE_BYTES;
                 uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
                 uint8_t *sF = sA + C::SF_OFF;
-                uint32_t *sfb = reinterpret_cast<uint32_t *>(sF + C::NUM_A * 512);
+                uint32_t *sfb = reinterpret_cast<uint32_t *>(sF + C::NUM_A * C::KPB * 512);
                 // activation scales in the block layout: column n at word
-                // (n % 32) * 4 + n / 32, its byte repeated for the 4 slices
-                for (int n = lane; n < BN; n += 32) {
-                    const uint32_t b = n < t.nrows ? (uint32_t)sxs[n * KBp + kb] : 127u;
-                    sfb[(n & 31) * 4 + (n >> 5)] = b * 0x01010101u;
-                }
+                // (n % 32) * 4 + n / 32 of its k-block's block, the byte
+                // repeated for the 4 slices
+#pragma unroll
+                for (int j = 0; j < C::KPB; ++j)
+                    for (int n = lane; n < BN; n += 32) {
+                        const uint32_t b = (n < t.nrows && j < nkb) ? (uint32_t)sxs[n * KBp + kb0 + j] : 127u;
+                        sfb[j * 128 + (n & 31) * 4 + (n >> 5)] = b * 0x01010101u;
+                    }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
+                    // boxes past the last k-block are zero-filled and still
+                    // counted; the E2M1 loads count their packed bytes
+                    const uint32_t bytes = C::NUM_A * (C::A_BYTES / 2 + nkb * 512) + C::B_BYTES;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     armed[stage] = (int)phase;
-                    tma_load_2d(sA, &tmA, &full[stage], kb * 128, arow, pol_w);
-                    bulk_load(sF, sfa0 + (size_t)kb * 512, 512, &full[stage], pol_w);
+                    tma_load_3d(sA, &tmA, &full[stage], 0, arow, kb0, pol_w);
+                    bulk_load(sF, sfa0 + (size_t)kb0 * 512, nkb * 512, &full[stage], pol_w);
                     if (GATE_UP) {
-                        tma_load_2d(sA + C::A_BYTES, &tmA, &full[stage], kb * 128,
-                                    arow + args.up_offset, pol_w);
-                        bulk_load(sF + 512, sfa1 + (size_t)kb * 512, 512, &full[stage], pol_w);
+                        tma_load_3d(sA + C::A_BYTES, &tmA, &full[stage], 0, arow + args.up_offset, kb0,
+                                    pol_w);
+                        bulk_load(sF + C::KPB * 512, sfa1 + (size_t)kb0 * 512, nkb * 512, &full[stage],
+                                  pol_w);
                     }
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sB + b * C::BOX * 128, &tmB, &full[stage], kb * 128,
-                                    t.row0 + b * C::BOX, pol_x);
+                    tma_load_3d(sB, &tmB, &full[stage], 0, t.row0, kb0, pol_x);
                 }
                 if (++stage == NST) { stage = 0; phase ^= 1; }
             }
@@ -215,40 +227,37 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                 if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
                     atomicOr(args.status, DEV_TIMEOUT);
         }
-    } else if (warp == 1) {
-        // --------------------------------------------------- MMA issue ----
+    } else if (warp == 1 || warp >= 2 + kEpiF) {
+        // ---------------------------------------------- MMA issue (A operand r) ----
+        const int r = warp == 1 ? 0 : 1;
         if (lane == 0) {
             int stage = 0, ab = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true;
-            const uint32_t tsf = tmem_base + C::SF_COL;       // A0 scales; A1 at +4; B at +4*NUM_A
-            const uint32_t tsfb = tsf + 4 * C::NUM_A;
+            const uint32_t tsfa = tmem_base + C::SF_COL + 4 * r;               // A scales
+            const uint32_t tsfb = tmem_base + C::SF_COL + 4 * C::NUM_A + 4 * r;  // B scales
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
                 const uint32_t idesc = idesc_mxf4_e4m3(kBM, (t.nrows + 15) & ~15);
                 if (!mbar_wait(&aempty[ab], aphase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d = tmem_base + ab * C::ACC;
-                for (int kb = 0; kb < KB; ++kb) {
+                const uint32_t d = tmem_base + ab * C::ACC + r * BN;
+                for (int kb0 = 0; kb0 < KB; kb0 += C::KPB) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(ring + stage * C::STAGE_BYTES);
                     const uint32_t sf = sa + C::SF_OFF;
-                    tmem_cp_32x128b_x4(tsf, sdesc_rows16(sf));
-                    if (GATE_UP) tmem_cp_32x128b_x4(tsf + 4, sdesc_rows16(sf + 512));
-                    tmem_cp_32x128b_x4(tsfb, sdesc_rows16(sf + C::NUM_A * 512));
-                    const uint64_t da = sdesc_sw128(sa);
-                    const uint64_t da2 = sdesc_sw128(sa + C::A_BYTES);
-                    const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES);
+                    for (int j = 0; j < C::KPB && kb0 + j < KB; ++j) {
+                        tmem_cp_32x128b_x4(tsfa, sdesc_rows16(sf + (r * C::KPB + j) * 512));
+                        tmem_cp_32x128b_x4(tsfb, sdesc_rows16(sf + (C::NUM_A * C::KPB + j) * 512));
+                        const uint64_t da = sdesc_sw128(sa + r * C::A_BYTES + j * C::A_KB);
+                        const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES + j * C::B_KB);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t id = idesc | idesc_sf_ids(k, k);
-                        const uint32_t sel = (uint32_t)k << 30;
-                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                        mma_mxf4_ss(d, da + 2 * k, db + 2 * k, id, tsf | sel, tsfb | sel, acc);
-                        if (GATE_UP)
-                            mma_mxf4_ss(d + BN, da2 + 2 * k, db + 2 * k, id, (tsf + 4) | sel,
-                                        tsfb | sel, acc);
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t sel = (uint32_t)k << 30;
+                            mma_mxf4_ss(d, da + 2 * k, db + 2 * k, idesc | idesc_sf_ids(k, k),
+                                        tsfa | sel, tsfb | sel, (kb0 + j > 0 || k > 0) ? 1u : 0u);
+                        }
                     }
                     mma_commit(&empty[stage]);
                     if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -386,22 +395,36 @@ cudaError_t launch_oneF(const CUtensorMap &a, const CUtensorMap &b, const GemmFA
         if (e != cudaSuccess) return e;
         attr_bytes[dev & 63] = need;
     }
-    return launch_k(grouped_gemm_mxf4<GATE_UP, BN>, dim3(num_sms()), dim3(kThreadsF), need, st, true,
+    return launch_k(grouped_gemm_mxf4<GATE_UP, BN>, dim3(num_sms()), dim3(C::THREADS), need, st, true,
                     a, b, af);
 }
 
-// Packed E2M1 matrix [rows][cols] (cols/2 bytes a row): boxes of 128 rows x
-// 128 elements, each 16 codes expanded to a 16-byte slot in shared memory,
-// 128-byte swizzle.
-bool make_tmap_e2m1(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols) {
+// A row-major [rows][cols] matrix seen as 3-D (k-element within a 128-block,
+// row, 128-block) so that one box brings `kpb` k-blocks of `box_rows` rows as
+// [k-block][row][128 bytes] tiles with the 128-byte swizzle.
+// Packed E2M1 (cols/2 bytes a row): each 16 codes land in a 16-byte slot.
+bool make_tmap_e2m1(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t kpb) {
     auto enc = tmap_encoder();
     if (!enc) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols / 2};
-    cuuint32_t box[2] = {128, (cuuint32_t)kBM};
-    cuuint32_t es[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void *>(ptr), dims, strides,
+    cuuint64_t dims[3] = {128, rows, cols / 128};
+    cuuint64_t strides[2] = {cols / 2, 64};
+    cuuint32_t box[3] = {128, (cuuint32_t)kBM, kpb};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(ptr), dims, strides,
                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// E4M3 activations [rows][cols] bytes, the same 3-D view.
+bool make_tmap_e4m3_kb(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows, uint32_t kpb) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, rows, cols / 128};
+    cuuint64_t strides[2] = {cols, 128};
+    cuuint32_t box[3] = {128, box_rows, kpb};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -413,14 +436,14 @@ cudaError_t launch_gemms_mxf4(const void *w13, const uint8_t *w13sf, const void 
                               cudaStream_t st) {
     if (H / 128 > kMaxKBF || F / 128 > kMaxKBF) return cudaErrorInvalidValue;
     if (bn != kBNFp8 && bn != kBNFp8Decode) return cudaErrorInvalidValue;
-    const int box = bn < 32 ? bn : 32;
     const uint64_t N = (uint64_t)T * K;
+    constexpr uint32_t kpb = CfgF<true, kBNFp8>::KPB;
+    static_assert(CfgF<true, kBNFp8>::KPB == CfgF<false, kBNFp8Decode>::KPB, "one k-block grouping");
     CUtensorMap ta, tb, tc, td;
-    const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    if (!make_tmap_e2m1(&ta, w13, (uint64_t)E * 2 * F, H) ||
-        !make_tmap(&tb, U8, 1, ws + L.xperm, N, H, box) ||
-        !make_tmap_e2m1(&tc, w2, (uint64_t)E * H, F) ||
-        !make_tmap(&td, U8, 1, ws + L.h, N, F, box))
+    if (!make_tmap_e2m1(&ta, w13, (uint64_t)E * 2 * F, H, kpb) ||
+        !make_tmap_e4m3_kb(&tb, ws + L.xperm, N, H, bn, kpb) ||
+        !make_tmap_e2m1(&tc, w2, (uint64_t)E * H, F, kpb) ||
+        !make_tmap_e4m3_kb(&td, ws + L.h, N, F, bn, kpb))
         return cudaErrorInvalidValue;
     GemmFArgs g = {};
     g.offsets = (const int32_t *)(ws + L.offsets);
