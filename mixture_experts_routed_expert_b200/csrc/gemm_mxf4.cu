@@ -20,11 +20,12 @@
 //     all four lane quarters) and issues four MMAs of K = 32 per k-block,
 //     each selecting its scale byte.
 // Tiles and epilogues as in the E4M3 kernel.  Warp roles: warp 0 TMA
-// producer, warp 1 TMEM allocation + MMA issue for the gate (or down) operand,
-// warps 2-9 epilogue from double-buffered TMEM accumulators, warp 10 (gate_up
-// only) MMA issue for the up operand: with a few routed rows per tile an MMA
-// instruction does little tensor work, and two issuing warps keep the tensor
-// cores fed where one could not.
+// producer, warps 1 and 10 MMA issue (warp 1 also allocates TMEM), warps 2-9
+// epilogue from double-buffered TMEM accumulators.  With a few routed rows per
+// tile an MMA instruction does little tensor work, and two issuing warps keep
+// the tensor cores fed where one could not: gate_up issues gate and up from
+// separate warps, down the two k-blocks of each stage into two partial
+// accumulators that the epilogue adds.
 //   S4 (gate_up): h = bf16(SiLU(g) * u), quantised per 128 features (the
 //     tile's rows) to E4M3 with a power-of-two scale -> hq [N][F] and the
 //     scale's E8M0 byte -> hsf [N][FBp].
@@ -49,9 +50,11 @@ template <bool GATE_UP, int BN>
 struct CfgF {
     static_assert(BN == 64 || BN == 16, "one epilogue thread owns 32 or 8 columns");
     static constexpr int NUM_A = GATE_UP ? 2 : 1;
-    // one MMA-issuing warp per A operand (gate, up): the issue of block-scaled
-    // MMAs with few routed rows, not the tensor cores, paces a k-block
-    static constexpr int THREADS = 64 + 32 * kEpiF + 32 * (NUM_A - 1);
+    // two MMA-issuing warps: the issue of block-scaled MMAs with few routed
+    // rows, not the tensor cores, paces a k-block.  gate_up: one per A operand
+    // (gate, up); down: one per k-block of a stage, each into its own partial
+    // accumulator (summed by the epilogue)
+    static constexpr int THREADS = 64 + 32 * kEpiF + 32;
     static constexpr int MAX_STAGES = 12;
     // k-blocks per pipeline stage: one 3-D TMA load per operand and stage, so
     // that the producer's issue cost per byte halves
@@ -62,9 +65,9 @@ struct CfgF {
     static constexpr int B_BYTES = KPB * B_KB;          // [kb][routed row][128]
     static constexpr int SF_OFF = NUM_A * A_BYTES + B_BYTES;   // scale blocks: [A0][A1][B] x KPB
     static constexpr int STAGE_BYTES = (SF_OFF + (NUM_A + 1) * KPB * 512 + 1023) / 1024 * 1024;
-    static constexpr int ACC = NUM_A * BN;              // TMEM columns of one accumulator set
+    static constexpr int ACC = 2 * BN;                  // TMEM columns of one accumulator set
     static constexpr int SF_COL = 2 * ACC;              // scale columns after the two sets
-    static constexpr int COLS_USED = SF_COL + 8 * NUM_A;   // per operand: A and B scale columns
+    static constexpr int COLS_USED = SF_COL + 16;       // per MMA warp: A and B scale columns
     static constexpr int TMEM_COLS =
         COLS_USED <= 64 ? 64 : (COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512));
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
@@ -130,10 +133,10 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], C::NUM_A);
+            mbar_init(&empty[s], 2);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&afull[b], C::NUM_A);
+            mbar_init(&afull[b], 2);
             mbar_init(&aempty[b], 32 * kEpiF);
         }
         *abort_flag = 0;
@@ -233,14 +236,18 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
                     atomicOr(args.status, DEV_TIMEOUT);
         }
     } else if (warp == 1 || warp >= 2 + kEpiF) {
-        // ---------------------------------------------- MMA issue (A operand r) ----
+        // ------------------------------------------------ MMA issue (role r) ----
+        // gate_up: A operand r, every k-block; down: A operand 0, the k-blocks
+        // j == r of each stage, into partial accumulator r
+        static_assert(GATE_UP || C::KPB == 2, "down splits each stage's two k-blocks");
         const int r = warp == 1 ? 0 : 1;
+        const int op = GATE_UP ? r : 0;
         if (lane == 0) {
             int stage = 0, ab = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true;
-            const uint32_t tsfa = tmem_base + C::SF_COL + 4 * r;               // A scales
-            const uint32_t tsfb = tmem_base + C::SF_COL + 4 * C::NUM_A + 4 * r;  // B scales
+            const uint32_t tsfa = tmem_base + C::SF_COL + 8 * r;      // A scales
+            const uint32_t tsfb = tsfa + 4;                            // B scales
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
                 const uint32_t idesc = idesc_mxf4_e4m3(kBM, (t.nrows + 15) & ~15);
@@ -253,15 +260,17 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
                     const uint32_t sa = smem_u32(ring + stage * C::STAGE_BYTES);
                     const uint32_t sf = sa + C::SF_OFF;
                     for (int j = 0; j < C::KPB && kb0 + j < KB; ++j) {
-                        tmem_cp_32x128b_x4(tsfa, sdesc_rows16(sf + (r * C::KPB + j) * 512));
+                        if (!GATE_UP && j != r) continue;
+                        tmem_cp_32x128b_x4(tsfa, sdesc_rows16(sf + (op * C::KPB + j) * 512));
                         tmem_cp_32x128b_x4(tsfb, sdesc_rows16(sf + (C::NUM_A * C::KPB + j) * 512));
-                        const uint64_t da = sdesc_sw128(sa + r * C::A_BYTES + j * C::A_KB);
+                        const uint64_t da = sdesc_sw128(sa + op * C::A_BYTES + j * C::A_KB);
                         const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES + j * C::B_KB);
+                        const int first = GATE_UP ? 0 : r;   // this role's first k-block
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint32_t sel = (uint32_t)k << 30;
                             mma_mxf4_ss(d, da + 2 * k, db + 2 * k, idesc | idesc_sf_ids(k, k),
-                                        tsfa | sel, tsfb | sel, (kb0 + j > 0 || k > 0) ? 1u : 0u);
+                                        tsfa | sel, tsfb | sel, (kb0 + j > first || k > 0) ? 1u : 0u);
                         }
                     }
                     mma_commit(&empty[stage]);
@@ -308,6 +317,11 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int j = 0; j < NC; ++j) au[j] = __uint_as_float(r[j]);
+                } else if (KB > 1) {                 // the second partial accumulator
+                    if constexpr (NC == 32) tmem_ld32(ta + BN, r); else tmem_ld8(ta + BN, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < NC; ++j) ag[j] += __uint_as_float(r[j]);
                 }
             }
             tc_fence_before();
