@@ -54,7 +54,10 @@ struct CfgF {
     // rows, not the tensor cores, paces a k-block.  gate_up: one per A operand
     // (gate, up); down: one per k-block of a stage, each into its own partial
     // accumulator (summed by the epilogue)
-    static constexpr int THREADS = 64 + 32 * kEpiF + 32;
+    // and two TMA-issuing warps (A operands on one side, activations and their
+    // scales on the other), for the same reason
+    static constexpr int MMA1 = 2 + kEpiF, PROD1 = 3 + kEpiF;   // warps 10 and 11
+    static constexpr int THREADS = 32 * (PROD1 + 1);
     static constexpr int MAX_STAGES = 12;
     // k-blocks per pipeline stage: one 3-D TMA load per operand and stage, so
     // that the producer's issue cost per byte halves
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = lane_id();
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 2);
             mbar_init(&empty[s], 2);
         }
         for (int b = 0; b < 2; ++b) {
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) {
+    if ((warp == 0 || warp == C::PROD1) && lane == 0) {
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
     }
@@ -162,8 +165,13 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
     const int total = s_tiles[args.E] * args.MT;
     pdl_launch_dependents();
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer ----
+    if (warp == 0 || warp == C::PROD1) {
+        // ------------------------------------------------ TMA producers ----
+        // producer p loads A operand p (if it exists); the activations and
+        // their scales come from producer 0 in gate_up and producer 1 in down
+        const int p = warp == 0 ? 0 : 1;
+        const bool do_a = p < C::NUM_A;
+        const bool do_b = GATE_UP ? p == 0 : p == 1;
         const uint64_t pol_once = policy_evict_first();
         const uint64_t pol_x = policy_evict_last();
         const int KBp = args.KBp;
@@ -173,19 +181,21 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
         bool ok = true;
         for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
             const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
-            // the tile's activation-scale bytes, row n -> sxs[n][0..KBp)
-            const int nch = KBp / 16;
-            for (int i = lane; i < t.nrows * nch; i += 32) {
-                const int n = i / nch, c = i - n * nch;
-                cp_async16(sxs + n * KBp + 16 * c, args.xsf + (size_t)(t.row0 + n) * KBp + 16 * c);
+            if (do_b) {
+                // the tile's activation-scale bytes, row n -> sxs[n][0..KBp)
+                const int nch = KBp / 16;
+                for (int i = lane; i < t.nrows * nch; i += 32) {
+                    const int n = i / nch, c = i - n * nch;
+                    cp_async16(sxs + n * KBp + 16 * c, args.xsf + (size_t)(t.row0 + n) * KBp + 16 * c);
+                }
+                cp_async_commit();
+                cp_async_wait<0>();
+                __syncwarp();
             }
-            cp_async_commit();
-            cp_async_wait<0>();
-            __syncwarp();
             const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
-            const int arow = t.e * args.a_rows_per_expert + t.m * kBM;
-            const uint8_t *sfa0 = args.wsf + t.e * args.wsf_per_expert + (size_t)t.m * KB * 512;
-            const uint8_t *sfa1 = sfa0 + (size_t)(args.up_offset / kBM) * KB * 512;
+            const int arow = t.e * args.a_rows_per_expert + t.m * kBM + p * args.up_offset;
+            const uint8_t *sfa = args.wsf + t.e * args.wsf_per_expert +
+                                 ((size_t)t.m + (size_t)p * (args.up_offset / kBM)) * KB * 512;
             for (int kb0 = 0; kb0 < KB; kb0 += C::KPB) {
                 const int nkb = min(C::KPB, KB - kb0);
                 if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag);
@@ -194,33 +204,33 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
                 uint8_t *sA = ring + stage * C::STAGE_BYTES;
                 uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
                 uint8_t *sF = sA + C::SF_OFF;
-                uint32_t *sfb = reinterpret_cast<uint32_t *>(sF + C::NUM_A * C::KPB * 512);
-                // activation scales in the block layout: column n at word
-                // (n % 32) * 4 + n / 32 of its k-block's block, the byte
-                // repeated for the 4 slices
+                if (do_b) {
+                    // activation scales in the block layout: column n at word
+                    // (n % 32) * 4 + n / 32 of its k-block's block, the byte
+                    // repeated for the 4 slices
+                    uint32_t *sfb = reinterpret_cast<uint32_t *>(sF + C::NUM_A * C::KPB * 512);
 #pragma unroll
-                for (int j = 0; j < C::KPB; ++j)
-                    for (int n = lane; n < BN; n += 32) {
-                        const uint32_t b = (n < t.nrows && j < nkb) ? (uint32_t)sxs[n * KBp + kb0 + j] : 127u;
-                        sfb[j * 128 + (n & 31) * 4 + (n >> 5)] = b * 0x01010101u;
-                    }
-                fence_proxy_async_smem();
+                    for (int j = 0; j < C::KPB; ++j)
+                        for (int n = lane; n < BN; n += 32) {
+                            const uint32_t b =
+                                (n < t.nrows && j < nkb) ? (uint32_t)sxs[n * KBp + kb0 + j] : 127u;
+                            sfb[j * 128 + (n & 31) * 4 + (n >> 5)] = b * 0x01010101u;
+                        }
+                    fence_proxy_async_smem();
+                }
                 __syncwarp();
                 if (lane == 0) {
                     // boxes past the last k-block are zero-filled and still
                     // counted; the E2M1 loads count their packed bytes
-                    const uint32_t bytes = C::NUM_A * (C::A_BYTES / 2 + nkb * 512) + C::B_BYTES;
+                    const uint32_t bytes = (do_a ? C::A_BYTES / 2 + nkb * 512 : 0) + (do_b ? C::B_BYTES : 0);
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     armed[stage] = (int)phase;
-                    tma_load_3d(sA, &tmA, &full[stage], 0, arow, kb0, pol_w);
-                    bulk_load(sF, sfa0 + (size_t)kb0 * 512, nkb * 512, &full[stage], pol_w);
-                    if (GATE_UP) {
-                        tma_load_3d(sA + C::A_BYTES, &tmA, &full[stage], 0, arow + args.up_offset, kb0,
-                                    pol_w);
-                        bulk_load(sF + C::KPB * 512, sfa1 + (size_t)kb0 * 512, nkb * 512, &full[stage],
+                    if (do_a) {
+                        tma_load_3d(sA + p * C::A_BYTES, &tmA, &full[stage], 0, arow, kb0, pol_w);
+                        bulk_load(sF + p * C::KPB * 512, sfa + (size_t)kb0 * 512, nkb * 512, &full[stage],
                                   pol_w);
                     }
-                    tma_load_3d(sB, &tmB, &full[stage], 0, t.row0, kb0, pol_x);
+                    if (do_b) tma_load_3d(sB, &tmB, &full[stage], 0, t.row0, kb0, pol_x);
                 }
                 if (++stage == NST) { stage = 0; phase ^= 1; }
             }
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
                 if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
                     atomicOr(args.status, DEV_TIMEOUT);
         }
-    } else if (warp == 1 || warp >= 2 + kEpiF) {
+    } else if (warp == 1 || warp == C::MMA1) {
         // ------------------------------------------------ MMA issue (role r) ----
         // gate_up: A operand r, every k-block; down: A operand 0, the k-blocks
         // j == r of each stage, into partial accumulator r
