@@ -153,7 +153,12 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
-    pdl_wait();
+    // gate_up reads the permutation's outputs, so it waits for the kernels
+    // before it.  down is launched only once gate_up, which waited for the
+    // permutation, runs: the offsets and tiles are final, and only the h rows
+    // and their scales (gate_up's outputs) need the wait, taken by the
+    // producer that loads them -- the weights start streaming at once.
+    if (GATE_UP) pdl_wait();
     for (int i = threadIdx.x; i <= args.E; i += blockDim.x) {
         s_off[i] = args.offsets[i];
         s_tiles[i] = args.tiles[i];
@@ -172,6 +177,7 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
         const int p = warp == 0 ? 0 : 1;
         const bool do_a = p < C::NUM_A;
         const bool do_b = GATE_UP ? p == 0 : p == 1;
+        if (!GATE_UP && do_b) pdl_wait();
         const uint64_t pol_once = policy_evict_first();
         const uint64_t pol_x = policy_evict_last();
         const int KBp = args.KBp;
