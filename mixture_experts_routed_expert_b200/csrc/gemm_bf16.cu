@@ -33,12 +33,15 @@ constexpr int kStages = 4;
 constexpr int kBK = 64;           // bf16 elements per k-block = one 128-byte swizzle row
 constexpr int kBoxRows = 32;      // routed rows per TMA box of the B operand
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
 
 template <bool GATE_UP>
 struct Cfg {
     static constexpr int BN = GATE_UP ? kBNGateUp : kBNDown;
     static constexpr int NUM_A = GATE_UP ? 2 : 1;      // gate and up weight tiles
+    // gate_up: one MMA-issuing warp per weight tile (warps 1 and 10): with
+    // 128-row tiles and up to 128 routed rows the issue of the MMAs, not the
+    // tensor pipe, paced a k-block when one warp issued both
+    static constexpr int THREADS = 64 + 32 * kEpiWarps + 32 * (NUM_A - 1);
     static constexpr int A_BYTES = kBM * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
@@ -68,7 +71,7 @@ struct GemmArgs {
 };
 
 template <bool GATE_UP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<GATE_UP>::THREADS, 1)
     grouped_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                       const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
     using C = Cfg<GATE_UP>;
@@ -90,10 +93,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], C::NUM_A);
         }
         for (int a = 0; a < C::NUM_ACC; ++a) {
-            mbar_init(&tfull[a], 1);
+            mbar_init(&tfull[a], C::NUM_A);
             mbar_init(&tempty[a], 32 * kEpiWarps);
         }
         *abort_flag = 0;
@@ -168,8 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
                     atomicOr(args.status, DEV_TIMEOUT);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 2 + kEpiWarps) {
         // ------------------------------------------------ MMA issuer ------
+        const int r = warp == 1 ? 0 : 1;          // weight tile (gate, up) of this warp
         if (lane == 0) {
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
@@ -180,20 +184,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t idesc = idesc_bf16(kBM, N);
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d = tmem_base + acc * C::ACC_COLS;
+                const uint32_t d = tmem_base + acc * C::ACC_COLS + r * C::BN;
                 for (int kb = 0; kb < args.KB; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(ring + stage * C::STAGE_BYTES);
-                    const uint64_t da = sdesc_sw128(sa);
-                    const uint64_t da2 = sdesc_sw128(sa + C::A_BYTES);
+                    const uint64_t da = sdesc_sw128(sa + r * C::A_BYTES);
                     const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        const uint32_t accum = (kb | k) != 0;
-                        mma_bf16_ss(d, da + 2 * k, db + 2 * k, idesc, accum);
-                        if (GATE_UP) mma_bf16_ss(d + C::BN, da2 + 2 * k, db + 2 * k, idesc, accum);
-                    }
+                    for (int k = 0; k < kBK / 16; ++k)
+                        mma_bf16_ss(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
                     mma_commit(&empty[stage]);
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
@@ -293,7 +293,7 @@ cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &a2, const CUtens
         if (e != cudaSuccess) return e;
         attr_done[dev & 63] = 1;
     }
-    return launch_k(grouped_gemm_bf16<GATE_UP>, dim3(num_sms()), dim3(kThreads), smem, st, true, a,
+    return launch_k(grouped_gemm_bf16<GATE_UP>, dim3(num_sms()), dim3(C::THREADS), smem, st, true, a,
                     a2, b, args);
 }
 
