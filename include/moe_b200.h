@@ -148,6 +148,28 @@ MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *g
                                 size_t workspace_bytes, void *stream);
 
 /*
+ * The MXFP4 decode form as one persistent kernel after the permutation
+ * (row "single-kernel fusion" of the DeepGEMM Mega MoE news page: the MoE
+ * steps in one kernel so that the intermediate round trips go away): gate_up
+ * tiles, down tiles and the top-K combine run in the same launch, the down
+ * tiles of a 16-row tile waiting (bounded) for its gate_up tiles, the last
+ * down tile of a (token, 128-row block) summing that block in k order.
+ * Same arguments, layouts and results as moe_experts_decode with
+ * wt = MOE_W_MXFP4 and T <= 16, T * K <= 64 (otherwise MOE_ERR_UNSUPPORTED);
+ * workspace from moe_experts_workspace_size(..., MOE_W_MXFP4, 1).  On B200 it
+ * is not faster than moe_experts_decode's separate kernels at these sizes
+ * (programmatic dependent launch already overlaps their boundaries, and each
+ * down tile needs all of its rows' gate_up tiles), so moe_experts_decode
+ * does not use it.
+ */
+MOE_API moe_status_t moe_experts_decode_fused(const void *hidden_states, const void *gate_up_proj,
+                                      const void *down_proj, const int32_t *top_k_index,
+                                      const float *top_k_weights, int top_k, int T, int H, int F,
+                                      int E, moe_wtype_t wt, const void *gate_up_scale,
+                                      const void *down_scale, void *out, void *workspace,
+                                      size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of workspace needed by moe_experts_with_shared for these sizes
  * (0 when the sizes are invalid).
  */

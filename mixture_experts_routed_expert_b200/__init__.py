@@ -26,7 +26,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "M
 EXPORTS = ("moe_abi_version", "moe_status_string", "moe_experts_workspace_size",
            "moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
            "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
-           "moe_experts_shared_workspace_size", "moe_experts_with_shared")
+           "moe_experts_shared_workspace_size", "moe_experts_with_shared",
+           "moe_experts_decode_fused")
 
 
 def _load():
@@ -43,6 +44,7 @@ def _load():
     fwd = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, Z, P]
     L.moe_experts_prefill.argtypes = fwd
     L.moe_experts_decode.argtypes = fwd
+    L.moe_experts_decode_fused.argtypes = fwd
     L.moe_route_sigmoid_grouped.argtypes = [P, P, I, I, I, I, I, F, P, P, P, P]
     L.quantize_fp8_block128.argtypes = [P, I, I, P, P, P]
     L.moe_debug_permute.argtypes = [P, I, I, I, P, P, P, P, P, Z, P]
@@ -52,7 +54,7 @@ def _load():
                                           P, P, P, P, I, P, P, P, Z, P]
     for n in ("moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
               "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
-              "moe_experts_with_shared"):
+              "moe_experts_with_shared", "moe_experts_decode_fused"):
         getattr(L, n).restype = I
     return L
 
@@ -121,7 +123,7 @@ def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_we
     wt = _wtype(gate_up_proj, weight_format)
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
-    decode = name == "moe_experts_decode"
+    decode = name in ("moe_experts_decode", "moe_experts_decode_fused")
     need = moe_experts_workspace_size(T, H, F2 // 2, E, top_k, wt, decode)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=hidden_states.device)
@@ -196,6 +198,16 @@ def moe_experts_with_shared(hidden_states, gate_up_proj, down_proj, top_k_index,
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc, "moe_experts_with_shared")
     return out
+
+
+def moe_experts_decode_fused(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
+                             top_k, gate_up_scale=None, down_scale=None, out=None, workspace=None,
+                             stream=None, weight_format="mxfp4"):
+    """MXFP4 decode form as one persistent kernel after the permutation
+    (gate_up, down and the combine in one launch); T <= 16, T*K <= 64."""
+    return _forward("moe_experts_decode_fused", hidden_states, gate_up_proj, down_proj,
+                    top_k_index, top_k_weights, top_k, gate_up_scale, down_scale, out, workspace,
+                    stream, weight_format)
 
 
 def moe_experts_decode_static(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,

@@ -64,6 +64,13 @@ Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t w
     Workspace L;
     Bump b;
     L.status = b.take(16);
+    // work counters of the fused MXFP4 decode kernel, next to the status word
+    // so that one clear covers both
+    L.ctr = L.status + 16;
+    L.ctr_bytes = (wt == MOE_W_MXFP4 && fused_mxf4_fits((int)T, K))
+                      ? sizeof(int32_t) * ((size_t)kFusedMaxSlots + (size_t)T * (H / 128))
+                      : 0;
+    b.off = align_up(L.ctr + L.ctr_bytes, 256);
     L.counts = b.take(sizeof(int32_t) * E);
     L.offsets = b.take(sizeof(int32_t) * (E + 1));
     L.tiles_g = b.take(sizeof(int32_t) * (E + 1));
@@ -319,6 +326,28 @@ moe_status_t moe_experts_with_shared(
                        wt, gate_up_scale, down_scale, out, workspace, SL.L.total, st,
                        wt == MOE_W_FP8_E4M3 && fp8_decode_sized(T, top_k) ? kBNFp8Decode : kBNFp8,
                        sh, residual);
+}
+
+moe_status_t moe_experts_decode_fused(const void *hidden_states, const void *gate_up_proj,
+                                      const void *down_proj, const int32_t *top_k_index,
+                                      const float *top_k_weights, int top_k, int T, int H, int F,
+                                      int E, moe_wtype_t wt, const void *gate_up_scale,
+                                      const void *down_scale, void *out, void *workspace,
+                                      size_t workspace_bytes, void *stream) {
+    moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                  top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
+                                  out);
+    if (s != MOE_OK || T == 0) return s;
+    if (wt != MOE_W_MXFP4 || !fused_mxf4_fits(T, top_k)) return MOE_ERR_UNSUPPORTED;
+    const Workspace L = prefill_workspace(T, H, F, E, top_k, wt);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return MOE_ERR_WORKSPACE;
+    return from_cuda(launch_fused_mxf4(hidden_states, gate_up_proj,
+                                       static_cast<const uint8_t *>(gate_up_scale), down_proj,
+                                       static_cast<const uint8_t *>(down_scale), top_k_index,
+                                       top_k_weights, T, H, F, E, top_k,
+                                       static_cast<uint8_t *>(workspace), L, out,
+                                       (cudaStream_t)stream));
 }
 
 moe_status_t moe_route_sigmoid_grouped(const float *logits, const float *bias, int T, int E,

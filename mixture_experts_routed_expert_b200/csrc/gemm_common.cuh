@@ -64,4 +64,34 @@ inline bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int elem_bytes, co
 }
 
 
+// A row-major [rows][cols] matrix seen as 3-D (k-element within a 128-block,
+// row, 128-block) so that one box brings `kpb` k-blocks of `box_rows` rows as
+// [k-block][row][128 bytes] tiles with the 128-byte swizzle.
+// Packed E2M1 (cols/2 bytes a row): each 16 codes land in a 16-byte slot.
+inline bool make_tmap_e2m1(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t kpb) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, rows, cols / 128};
+    cuuint64_t strides[2] = {cols / 2, 64};
+    cuuint32_t box[3] = {128, 128, kpb};   // 128 weight rows (one MMA tile)
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void *>(ptr), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// E4M3 activations [rows][cols] bytes, the same 3-D view.
+inline bool make_tmap_e4m3_kb(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows, uint32_t kpb) {
+    auto enc = tmap_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, rows, cols / 128};
+    cuuint64_t strides[2] = {cols, 128};
+    cuuint32_t box[3] = {128, box_rows, kpb};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+
 }  // namespace moe

@@ -21,6 +21,8 @@ constexpr int kBNFp8Decode = 16;  // the same GEMMs for a few tokens (decode ent
 // ---- workspace layout ------------------------------------------------------
 struct Workspace {
     size_t status;        // int32 device status word
+    size_t ctr;           // fused MXFP4 decode: int32 work counters (cleared with the status word)
+    size_t ctr_bytes;
     size_t counts;        // [E] int32
     size_t offsets;       // [E+1] int32
     size_t tiles_g;       // [E+1] int32 prefix of gate_up row tiles per expert
@@ -47,6 +49,8 @@ DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t 
 
 constexpr int kDecodeMaxSlots = 64;  // T*K served by the decode kernels
 constexpr int kDecodeMaxT = 16;
+constexpr int kFusedMaxSlots = 64;   // T*K served by the fused MXFP4 decode kernel
+constexpr int kFusedMaxT = 16;
 
 // Host-side argument checks of the forward entry points (MOE_OK when valid).
 moe_status_t validate_forward(const void *x, const void *gu, const void *dn, const int32_t *idx,
@@ -70,9 +74,11 @@ int num_sms();
 
 cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, int bn_g, int bn_d,
                            uint8_t *ws, const Workspace &L, cudaStream_t st);
+// zero / nzero (MXFP4 only): int32 counters that the kernel also clears.
 cudaError_t launch_permute_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H,
                                   int E, int bn_g, int bn_d, moe_wtype_t wt, uint8_t *ws,
-                                  const Workspace &L, cudaStream_t st);
+                                  const Workspace &L, cudaStream_t st, int32_t *zero = nullptr,
+                                  int nzero = 0);
 cudaError_t launch_debug_outputs(const int32_t *idx, int64_t n_slots, int E, const uint8_t *ws,
                                  const Workspace &L, int32_t *counts, int32_t *offsets,
                                  int32_t *perm, int32_t *inv, cudaStream_t st);
@@ -86,6 +92,13 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
                              uint8_t *ws, const Workspace &L, cudaStream_t st,
                              const SharedSet &sh = SharedSet());
 // residual: optional [T][H] bf16 added after the slot sum (nullptr: none).
+// The fused MXFP4 decode kernel (one launch for T <= kFusedMaxT,
+// T*K <= kFusedMaxSlots): counters, h and y in the workspace L.
+bool fused_mxf4_fits(int T, int K);
+cudaError_t launch_fused_mxf4(const void *x, const void *w13, const uint8_t *w13sf, const void *w2,
+                              const uint8_t *w2sf, const int32_t *idx, const float *w, int T, int H,
+                              int F, int E, int K, uint8_t *ws, const Workspace &L, void *out,
+                              cudaStream_t st);
 // MXFP4 weights (packed E2M1 + E8M0 scales in the block layout), E4M3
 // activations with E8M0 scale bytes in the workspace's scale regions.
 cudaError_t launch_gemms_mxf4(const void *w13, const uint8_t *w13sf, const void *w2,

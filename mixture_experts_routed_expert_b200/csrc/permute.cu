@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
     int bn_d, const uint4 *__restrict__ x, void *__restrict__ xperm, float *__restrict__ xscale,
     int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ tiles_g,
     int32_t *__restrict__ tiles_d, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
-    int32_t *__restrict__ status) {
+    int32_t *__restrict__ status, int32_t *__restrict__ zero, int nzero) {
     extern __shared__ int32_t psm[];
     int32_t *cnt_all = psm;                 // [E+1] -> exclusive offsets
     int32_t *cnt_bef = cnt_all + (E + 1);   // [E] slots of e before this chunk
@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
             *status = 0;
             offsets[E] = total;
         }
+        for (int i = t; i < nzero; i += kPThreads) zero[i] = 0;   // consumers' work counters
         for (int i = t; i < E; i += kPThreads) offsets[i] = cnt_all[i];
         for (int p = total + t; p < n_slots; p += kPThreads) perm[p] = -1;
         // row-tile prefixes for both GEMMs
@@ -284,7 +285,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
 
 template <int MODE>
 cudaError_t launch_pg(const void *x, const int32_t *idx, int64_t n_slots, int K, int H, int E,
-                      int bn_g, int bn_d, uint8_t *ws, const Workspace &L, cudaStream_t st) {
+                      int bn_g, int bn_d, uint8_t *ws, const Workspace &L, cudaStream_t st,
+                      int32_t *zero = nullptr, int nzero = 0) {
     const size_t smem = sizeof(int32_t) * ((3 + kPWarps) * (size_t)E + 2);
     static int attr_done[64] = {};
     int dev = 0;
@@ -312,7 +314,7 @@ cudaError_t launch_pg(const void *x, const int32_t *idx, int64_t n_slots, int K,
                     (void *)(ws + L.xperm), (float *)(ws + L.xscale), (int32_t *)(ws + L.counts),
                     (int32_t *)(ws + L.offsets), (int32_t *)(ws + L.tiles_g),
                     (int32_t *)(ws + L.tiles_d), (int32_t *)(ws + L.perm), (int32_t *)(ws + L.inv),
-                    (int32_t *)(ws + L.status));
+                    (int32_t *)(ws + L.status), zero, nzero);
 }
 
 }  // namespace
@@ -324,9 +326,10 @@ cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, int bn_g,
 
 cudaError_t launch_permute_gather(const void *x, const int32_t *idx, int64_t n_slots, int K, int H,
                                   int E, int bn_g, int bn_d, moe_wtype_t wt, uint8_t *ws,
-                                  const Workspace &L, cudaStream_t st) {
+                                  const Workspace &L, cudaStream_t st, int32_t *zero, int nzero) {
     if (wt == MOE_W_BF16) return launch_pg<1>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
-    if (wt == MOE_W_MXFP4) return launch_pg<3>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
+    if (wt == MOE_W_MXFP4)
+        return launch_pg<3>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st, zero, nzero);
     return launch_pg<2>(x, idx, n_slots, K, H, E, bn_g, bn_d, ws, L, st);
 }
 

@@ -4,7 +4,8 @@ block-128 scales; block-scaled tcgen05 MMAs) against the oracle: full
 outputs on reduced shapes spanning several k-blocks, tiles and ragged tails,
 Zipf-skewed routing with empty experts, both tile heights (16-row tiles of
 decode-sized calls, 64-row tiles otherwise), and sampled tokens of the
-DeepSeek-V3-like layer (H=7168, F=2048, E=256, K=8) with MXFP4 weights."""
+DeepSeek-V3-like layer (H=7168, F=2048, E=256, K=8) with MXFP4 weights; the
+one-kernel decode form (moe_experts_decode_fused) on the same checks."""
 import pytest
 import torch
 
@@ -127,3 +128,54 @@ def test_mxf4_dsv3_sampled(moe, cuda_dev, dsv3_mxf4, T, fn):
     tokens = sorted({0, T // 2, T - 1})
     ref = _oracle(lay.x, dsv3_mxf4, idx, w, D["E"], tokens=tokens)
     assert_matches_oracle(out[tokens], ref, "mxf4 dsv3 T=%d" % T)
+
+
+# ------------------------------------------- one-kernel form (decode sizes) ----
+
+@pytest.mark.parametrize("T,H,F,E,K", [
+    (1, 512, 256, 16, 8),        # one token
+    (8, 640, 384, 32, 8),        # 64 slots; odd k-block counts (5 and 3)
+    (5, 384, 128, 16, 4),        # down with one k-block (one partial accumulator)
+    (16, 256, 256, 8, 4),        # 16 tokens, experts with > 16 slots (two row tiles)
+])
+def test_mxf4_fused_reduced_shapes(moe, cuda_dev, T, H, F, E, K):
+    lay = inputs.fp8_layer(T, seed=50 + T, H=H, F=F, E=E, weights=(None, None, None, None))
+    wts = inputs.mxf4_weights(seed=T + 1, H=H, F=F, E=E)
+    idx, w = _route(lay, K)
+    out = _run(moe, lay.x, wts, idx, w, cuda_dev, "moe_experts_decode_fused")
+    assert_matches_oracle(out, _oracle(lay.x, wts, idx, w, E), "fused T=%d" % T)
+
+
+def test_mxf4_fused_invalid_ids_and_empty_tokens(moe, cuda_dev):
+    T, H, F, E, K = 6, 256, 256, 8, 4
+    lay = inputs.fp8_layer(T, seed=9, H=H, F=F, E=E, weights=(None, None, None, None))
+    wts = inputs.mxf4_weights(seed=9, H=H, F=F, E=E)
+    idx, w = _route(lay, K)
+    idx[0, :] = 2                       # every slot of a token on one expert
+    idx[1, 3] = -1
+    idx[2, 0] = E
+    idx[4, :] = -7                      # a token with no valid slot -> 0
+    out = _run(moe, lay.x, wts, idx, w, cuda_dev, "moe_experts_decode_fused")
+    assert_matches_oracle(out, _oracle(lay.x, wts, idx, w, E), "fused invalid ids")
+    assert torch.all(out[4] == 0)
+    # nothing valid at all
+    idx_none = torch.full_like(idx, -1)
+    out = _run(moe, lay.x, wts, idx_none, w, cuda_dev, "moe_experts_decode_fused")
+    assert torch.all(out == 0)
+
+
+def test_mxf4_fused_deterministic_and_limits(moe, cuda_dev, dsv3_mxf4):
+    D = inputs.DSV3_FP8
+    lay = inputs.fp8_layer(8, seed=77, device=cuda_dev, weights=(None, None, None, None))
+    idx, w = _route(lay, D["K"])
+    a = _run(moe, lay.x, dsv3_mxf4, idx, w, cuda_dev, "moe_experts_decode_fused")
+    b = _run(moe, lay.x, dsv3_mxf4, idx, w, cuda_dev, "moe_experts_decode_fused")
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    ref = _oracle(lay.x, dsv3_mxf4, idx, w, D["E"], tokens=[0, 7])
+    assert_matches_oracle(a[[0, 7]], ref, "fused dsv3 T=8")
+    # 17 tokens is outside the one-kernel form
+    lay17 = inputs.fp8_layer(17, seed=3, H=256, F=256, E=8, weights=(None, None, None, None))
+    wts = inputs.mxf4_weights(seed=3, H=256, F=256, E=8)
+    idx17, w17 = _route(lay17, 2)
+    with pytest.raises(moe.MoEError):
+        _run(moe, lay17.x, wts, idx17, w17, cuda_dev, "moe_experts_decode_fused")
