@@ -484,7 +484,7 @@ def run_ours(args):
     mx_w = inputs.mxf4_weights(seed=0, device=dev)
     per_expert_mxf4 = 3 * D["F"] * D["H"] // 2 + 3 * D["F"] * D["H"] // 32
 
-    def mxf4_entry(T, zipf, steps):
+    def mxf4_entry(T, zipf, steps, fused=False):
         lay = inputs.fp8_layer(T, seed=T, device=dev, weights=(None, None, None, None), zipf=zipf)
         idx = torch.empty(T, D["K"], dtype=torch.int32, device=dev)
         tw = torch.empty(T, D["K"], dtype=torch.float32, device=dev)
@@ -493,6 +493,8 @@ def run_ours(args):
         wsz = moe.moe_experts_workspace_size(T, D["H"], D["F"], D["E"], D["K"], moe.MOE_W_MXFP4, dec)
         ws = torch.empty(wsz, dtype=torch.uint8, device=dev)
         fn = moe.moe_experts_decode if dec else moe.moe_experts_prefill
+        if fused:
+            fn = moe.moe_experts_decode_fused
 
         def call():
             moe.moe_route_sigmoid_grouped(lay.logits, lay.bias, D["num_groups"], D["topk_group"],
@@ -516,6 +518,9 @@ def run_ours(args):
 
     for T in (128, 8, 1):
         breakdown["mxf4_dsv3_T%d" % T] = mxf4_entry(T, None, args.steps)
+    for T in (8, 1):   # the same calls through the one-kernel form
+        breakdown["mxf4_dsv3_fused_T%d" % T] = dict(mxf4_entry(T, None, args.steps, fused=True),
+                                                    entry="decode_fused")
     # skewed sweep (Zipf 1.1 expert popularity), FP8 and the OCR-2 bf16 shape
     sweep_steps = max(3, min(args.steps, 10))
     sweep = {}
