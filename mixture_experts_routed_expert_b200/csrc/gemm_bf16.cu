@@ -31,7 +31,11 @@ namespace {
 
 constexpr int kStages = 4;
 constexpr int kBK = 64;           // bf16 elements per k-block = one 128-byte swizzle row
-constexpr int kBoxRows = 32;      // routed rows per TMA box of the B operand
+// Routed rows per TMA box of the B operand, chosen at launch: 128 when the
+// experts average >= 64 routed rows (one TMA per k-block; 32-row boxes paced
+// the producer: T=2048 / 8192 layers 5 / 13 % slower), 32 for a few rows per
+// expert (128-row boxes fetch unused rows: T=4 / 8 decode 12 / 19 % slower).
+constexpr int kBoxRowsFew = 32, kBoxRowsMany = 128;
 constexpr int kEpiWarps = 8;
 
 template <bool GATE_UP>
@@ -68,6 +72,7 @@ struct GemmArgs {
     const int32_t *perm;         // [N] routed row -> slot
     const float *topw;           // [T*K] router weights
     int32_t *status;
+    int box_rows;                // routed rows per B box (kBoxRowsFew or kBoxRowsMany)
 };
 
 template <bool GATE_UP>
@@ -140,8 +145,9 @@ __global__ void __launch_bounds__(Cfg<GATE_UP>::THREADS, 1)
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, C::BN);
                 const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
-                const int nbox = (t.nrows + kBoxRows - 1) / kBoxRows;
-                const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * kBoxRows * 128;
+                const int box_rows = args.box_rows;
+                const int nbox = (t.nrows + box_rows - 1) / box_rows;
+                const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * box_rows * 128;
                 const bool second = t.e >= args.E_split;
                 const CUtensorMap *mA = second ? &tmA2 : &tmA;
                 const int arow = (second ? t.e - args.E_split : t.e) * args.a_rows_per_expert + t.m * kBM;
@@ -156,8 +162,8 @@ __global__ void __launch_bounds__(Cfg<GATE_UP>::THREADS, 1)
                         tma_load_2d(sA + C::A_BYTES, mA, &full[stage], kb * kBK,
                                     arow + args.up_offset, pol_w);
                     for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sB + b * kBoxRows * 128, &tmB, &full[stage], kb * kBK,
-                                    t.row0 + b * kBoxRows, pol_x);
+                        tma_load_2d(sB + b * box_rows * 128, &tmB, &full[stage], kb * kBK,
+                                    t.row0 + b * box_rows, pol_x);
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
             }
@@ -303,13 +309,14 @@ cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float
                               int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
                               cudaStream_t st, const SharedSet &sh) {
     const uint64_t N = (uint64_t)T * K;
+    const int box_rows = N >= (uint64_t)64 * E ? kBoxRowsMany : kBoxRowsFew;
     CUtensorMap ta, tb, tc, td, ta2, tc2;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int E_split = E - sh.S;  // routed experts; ids E_split.. are the shared set
     if (!make_tmap(&ta, BF, 2, gate_up, (uint64_t)E_split * 2 * F, H, kBM) ||
-        !make_tmap(&tb, BF, 2, ws + L.xperm, N, H, kBoxRows) ||
+        !make_tmap(&tb, BF, 2, ws + L.xperm, N, H, box_rows) ||
         !make_tmap(&tc, BF, 2, down, (uint64_t)E_split * H, F, kBM) ||
-        !make_tmap(&td, BF, 2, ws + L.h, N, F, kBoxRows))
+        !make_tmap(&td, BF, 2, ws + L.h, N, F, box_rows))
         return cudaErrorInvalidValue;
     if (sh.S > 0) {
         if (!make_tmap(&ta2, BF, 2, sh.gate_up, (uint64_t)sh.S * 2 * F, H, kBM) ||
@@ -323,6 +330,7 @@ cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float
     g.offsets = (const int32_t *)(ws + L.offsets);
     g.E = E;
     g.E_split = E_split;
+    g.box_rows = box_rows;
     g.perm = (const int32_t *)(ws + L.perm);
     g.topw = topw;
     g.status = (int32_t *)(ws + L.status);
