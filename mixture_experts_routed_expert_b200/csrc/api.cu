@@ -119,13 +119,14 @@ bool decode_serves(int T, int K, int H, int F, moe_wtype_t wt) {
     return wt == MOE_W_BF16 && T * K <= kGemvMaxSlots && decode_fits(T, K, H, F);
 }
 // Tile height of the E4M3 and MXFP4 grouped GEMMs: 16 routed rows for
-// decode-sized calls and whenever the experts average <= 8 routed rows (a
-// 64-row tile then loads and multiplies mostly unused rows; DeepSeek-V3-like
-// layer, T=128: E4M3 1267 -> 1177 us, MXFP4 857 -> 731 us; at 16 rows per
-// expert, T=512, 64-row tiles are 27-37 % faster).
+// decode-sized calls and whenever the experts average <= 6 routed rows (a
+// 64-row tile then loads and multiplies mostly unused rows).  DeepSeek-V3-like
+// layer, E4M3 / MXFP4, 16-row vs 64-row tiles: 4 rows per expert (T=128)
+// 1177 / 731 vs 1267 / 857 us; 8 rows (T=256) 1562 / 968 vs 1453 / 961 us;
+// 12 rows (T=384) 2004 / 1239 vs 1621 / 1082 us.
 int tile_rows_8(int64_t T, int K, int E) {
     const int64_t n = T * K;
-    return (n <= kDecodeMaxSlots || n <= (int64_t)8 * E) ? kBNFp8Decode : kBNFp8;
+    return (n <= kDecodeMaxSlots || n <= (int64_t)6 * E) ? kBNFp8Decode : kBNFp8;
 }
 
 moe_status_t check_common(const void *x, const void *gu, const void *dn, const int32_t *idx,
