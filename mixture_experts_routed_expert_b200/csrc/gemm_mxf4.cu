@@ -48,7 +48,7 @@ constexpr int KPB16 = 2;
 
 template <bool GATE_UP, int BN>
 struct CfgF {
-    static_assert(BN == 64 || BN == 16, "one epilogue thread owns 32 or 8 columns");
+    static_assert(BN == 16 || BN == 64 || BN == 112, "tile heights of the launcher");
     static constexpr int NUM_A = GATE_UP ? 2 : 1;
     // two MMA-issuing warps: the issue of block-scaled MMAs with few routed
     // rows, not the tensor cores, paces a k-block.  gate_up: one per A operand
@@ -102,6 +102,18 @@ struct GemmFArgs {
 
 __device__ __forceinline__ void epi_sync_f() {
     asm volatile("bar.sync 2, %0;" ::"n"(32 * kEpiF) : "memory");
+}
+
+// CS (8, 16, 24 or 32, warp-uniform) consecutive TMEM columns of this warp's
+// lanes into r[0..CS).
+__device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&r)[32], int CS) {
+    if (CS == 32) {
+        tmem_ld32(taddr, r);
+    } else {
+        if (CS & 16) tmem_ld16(taddr, r);
+        if (CS & 8) tmem_ld8(taddr + (CS & 16), *reinterpret_cast<uint32_t(*)[8]>(r + (CS & 16)));
+    }
+    tmem_ld_wait();
 }
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -313,7 +325,6 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
         bool ok = true;
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
-            const int live = t.nrows - half * NC;   // columns of this thread that hold routed rows
             if (ok && !mbar_wait(&afull[ab], aphase, abort_flag)) {
                 ok = false;
                 *abort_flag = 1;
@@ -321,40 +332,41 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
             }
             tc_fence_after();
             const uint32_t ta = tmem_base + ((uint32_t)(eg * 32) << 16) + ab * C::ACC + half * NC;
-            float ag[NC], au[GATE_UP ? NC : 1];
-            {
-                uint32_t r[NC];
-                if constexpr (NC == 32) tmem_ld32(ta, r); else tmem_ld8(ta, r);
-                tmem_ld_wait();
+            // this thread's NC columns in chunks of up to 32: TMEM -> registers,
+            // then h (gate_up) or y (down); the accumulator set goes back to
+            // the MMA warps once the last chunk is loaded
 #pragma unroll
-                for (int j = 0; j < NC; ++j) ag[j] = __uint_as_float(r[j]);
-                if (GATE_UP) {
-                    if constexpr (NC == 32) tmem_ld32(ta + BN, r); else tmem_ld8(ta + BN, r);
-                    tmem_ld_wait();
+            for (int c0 = 0; c0 < NC; c0 += 32) {
+                const int CS = NC - c0 < 32 ? NC - c0 : 32;
+                float ag[32], au[32];
+                {
+                    uint32_t r[32];
+                    load_cols(ta + c0, r, CS);
 #pragma unroll
-                    for (int j = 0; j < NC; ++j) au[j] = __uint_as_float(r[j]);
-                } else if (KB > 1) {                 // the second partial accumulator
-                    if constexpr (NC == 32) tmem_ld32(ta + BN, r); else tmem_ld8(ta + BN, r);
-                    tmem_ld_wait();
+                    for (int j = 0; j < 32; ++j) ag[j] = j < CS ? __uint_as_float(r[j]) : 0.f;
+                    if (GATE_UP || KB > 1) {         // up, or down's second partial accumulator
+                        load_cols(ta + BN + c0, r, CS);
 #pragma unroll
-                    for (int j = 0; j < NC; ++j) ag[j] += __uint_as_float(r[j]);
+                        for (int j = 0; j < 32; ++j) {
+                            const float v = j < CS ? __uint_as_float(r[j]) : 0.f;
+                            if (GATE_UP) au[j] = v; else ag[j] += v;
+                        }
+                    }
                 }
-            }
-            tc_fence_before();
-            mbar_arrive(&aempty[ab]);
-            if (++ab == 2) { ab = 0; aphase ^= 1; }
-            if (GATE_UP) {
-                // h = bf16(SiLU(g) * u) for this row (feature) and NC routed rows
+                if (c0 + 32 >= NC) {
+                    tc_fence_before();
+                    mbar_arrive(&aempty[ab]);
+                }
+                const int cbase = half * NC + c0;        // first tile column of this chunk
+                if (GATE_UP) {
+                    // h = bf16(SiLU(g) * u) for this row (feature) and CS routed rows
 #pragma unroll
-                for (int j = 0; j < NC; ++j)
-                    ag[j] = __bfloat162float(__float2bfloat16_rn(silu_f(ag[j]) * au[j]));
-                // column max of |h| over this warp's 32 rows: lane l ends
-                // with column l of each group of 32
-#pragma unroll
-                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
+                    for (int j = 0; j < 32; ++j)
+                        ag[j] = __bfloat162float(__float2bfloat16_rn(silu_f(ag[j]) * au[j]));
+                    // column max of |h| over this warp's 32 rows: lane l ends with column l
                     float v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = 32 * grp + j < NC ? fabsf(ag[32 * grp + j]) : 0.f;
+                    for (int j = 0; j < 32; ++j) v[j] = j < CS ? fabsf(ag[j]) : 0.f;
 #pragma unroll
                     for (int o = 16; o >= 1; o >>= 1) {
 #pragma unroll
@@ -365,42 +377,38 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
                             v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
                         }
                     }
-                    if (32 * grp + lane < NC) amax_s[eg * BN + half * NC + 32 * grp + lane] = v[0];
-                }
-                epi_sync_f();
-                if (et < BN) {
-                    const float m = fmaxf(fmaxf(amax_s[et], amax_s[BN + et]),
-                                          fmaxf(amax_s[2 * BN + et], amax_s[3 * BN + et]));
-                    const int k = fp8_block_exp(m);
-                    scale_s[et] = pow2f(-k);
-                    if (et < t.nrows)
-                        args.hsf[(size_t)(t.row0 + et) * args.FBp + t.m] = (uint8_t)(k + 127);
-                }
-                epi_sync_f();
-                uint8_t *hp = args.hq + (size_t)(t.row0 + half * NC) * args.F + t.m * kBM + row;
+                    if (lane < CS) amax_s[eg * BN + cbase + lane] = v[0];
+                    epi_sync_f();
+                    if (et < 2 * CS) {                  // one thread per column of the chunk
+                        const int col = (et / CS) * NC + c0 + et % CS;
+                        const float m = fmaxf(fmaxf(amax_s[col], amax_s[BN + col]),
+                                              fmaxf(amax_s[2 * BN + col], amax_s[3 * BN + col]));
+                        const int k = fp8_block_exp(m);
+                        scale_s[col] = pow2f(-k);
+                        if (col < t.nrows)
+                            args.hsf[(size_t)(t.row0 + col) * args.FBp + t.m] = (uint8_t)(k + 127);
+                    }
+                    epi_sync_f();
+                    uint8_t *hp = args.hq + (size_t)(t.row0 + cbase) * args.F + t.m * kBM + row;
 #pragma unroll
-                for (int j = 0; j < NC; ++j) {
-                    if (j < live)
-                        hp[(size_t)j * args.F] =
-                            (uint8_t)(e4m3x2(ag[j] * scale_s[half * NC + j], 0.f) & 0xFF);
-                }
-                epi_sync_f();                    // scale_s is rewritten by the next tile
-            } else {
-                float *yp = args.y + t.m * kBM + row;
-#pragma unroll
-                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
-                    const int c = half * NC + 32 * grp + lane;
-                    const int my_slot = (c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
-                    const float my_w = (c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
+                    for (int j = 0; j < 32; ++j)
+                        if (j < CS && cbase + j < t.nrows)
+                            hp[(size_t)j * args.F] = (uint8_t)(e4m3x2(ag[j] * scale_s[cbase + j], 0.f) & 0xFF);
+                } else {
+                    float *yp = args.y + t.m * kBM + row;
+                    const int c = cbase + lane;
+                    const int my_slot = (lane < CS && c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
+                    const float my_w = (lane < CS && c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
                         const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
-                        if (32 * grp + j < NC && 32 * grp + j < live)
-                            yp[(size_t)slot * args.H] = wj * ag[32 * grp + j];
+                        if (j < CS && cbase + j < t.nrows) yp[(size_t)slot * args.H] = wj * ag[j];
                     }
                 }
             }
+            if (++ab == 2) { ab = 0; aphase ^= 1; }
+            if (GATE_UP) epi_sync_f();               // amax_s / scale_s are rewritten by the next tile
         }
     }
     tc_fence_before();
@@ -441,9 +449,10 @@ cudaError_t launch_gemms_mxf4(const void *w13, const uint8_t *w13sf, const void 
                               int E, int K, int bn, uint8_t *ws, const Workspace &L,
                               cudaStream_t st) {
     if (H / 128 > kMaxKBF || F / 128 > kMaxKBF) return cudaErrorInvalidValue;
-    if (bn != kBNFp8 && bn != kBNFp8Decode) return cudaErrorInvalidValue;
+    if (bn != kBNFp8 && bn != kBNFp8Decode && bn != kBNMxf4Wide) return cudaErrorInvalidValue;
     const uint64_t N = (uint64_t)T * K;
-    const uint32_t kpb = bn == kBNFp8 ? CfgF<true, kBNFp8>::KPB : CfgF<true, kBNFp8Decode>::KPB;
+    const uint32_t kpb = bn == kBNFp8Decode ? CfgF<true, kBNFp8Decode>::KPB : CfgF<true, kBNFp8>::KPB;
+    static_assert(CfgF<true, kBNFp8>::KPB == CfgF<true, kBNMxf4Wide>::KPB, "one map per height group");
     CUtensorMap ta, tb, tc, td;
     if (!make_tmap_e2m1(&ta, w13, (uint64_t)E * 2 * F, H, kpb) ||
         !make_tmap_e4m3_kb(&tb, ws + L.xperm, N, H, bn, kpb) ||
@@ -488,6 +497,11 @@ cudaError_t launch_gemms_mxf4(const void *w13, const uint8_t *w13sf, const void 
         const cudaError_t err = launch_oneF<true, kBNFp8Decode>(ta, tb, a1, st);
         if (err != cudaSuccess) return err;
         return launch_oneF<false, kBNFp8Decode>(tc, td, a2, st);
+    }
+    if (bn == kBNMxf4Wide) {
+        const cudaError_t err = launch_oneF<true, kBNMxf4Wide>(ta, tb, a1, st);
+        if (err != cudaSuccess) return err;
+        return launch_oneF<false, kBNMxf4Wide>(tc, td, a2, st);
     }
     const cudaError_t err = launch_oneF<true, kBNFp8>(ta, tb, a1, st);
     if (err != cudaSuccess) return err;

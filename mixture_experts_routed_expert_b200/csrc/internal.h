@@ -17,6 +17,7 @@ constexpr int kBNGateUp = 128;    // routed rows (tokens) per gate_up tile
 constexpr int kBNDown = 256;      // routed rows per down tile
 constexpr int kBNFp8 = 64;        // routed rows per tile of both E4M3 GEMMs
 constexpr int kBNFp8Decode = 16;  // the same GEMMs for a few tokens (decode entry)
+constexpr int kBNMxf4Wide = 112;  // MXFP4 GEMMs with many routed rows per expert
 
 // ---- workspace layout ------------------------------------------------------
 struct Workspace {

@@ -2,8 +2,9 @@
 one E8M0 scale per row and 32 columns, E4M3 activations with power-of-two
 block-128 scales; block-scaled tcgen05 MMAs) against the oracle: full
 outputs on reduced shapes spanning several k-blocks, tiles and ragged tails,
-Zipf-skewed routing with empty experts, both tile heights (16-row tiles of
-decode-sized calls, 64-row tiles otherwise), and sampled tokens of the
+Zipf-skewed routing with empty experts, all three tile heights (16-row
+tiles for few routed rows per expert, 112-row tiles for many, 64-row tiles
+between), and sampled tokens of the
 DeepSeek-V3-like layer (H=7168, F=2048, E=256, K=8) with MXFP4 weights; the
 one-kernel decode form (moe_experts_decode_fused) on the same checks."""
 import pytest
@@ -55,8 +56,9 @@ def _run(moe, x, wts, idx, w, dev, fn="moe_experts_prefill"):
 @pytest.mark.parametrize("T,H,F,E,K,skew,fn", [
     (40, 256, 256, 8, 2, None, "moe_experts_prefill"),     # two k-blocks, several tiles
     (300, 1024, 512, 64, 8, None, "moe_experts_prefill"),  # ragged row tiles, 8 k-blocks
-    (512, 384, 384, 64, 8, 1.1, "moe_experts_prefill"),    # Zipf skew: empty / hot experts
-    (3, 512, 256, 16, 4, None, "moe_experts_prefill"),     # tiny T, 64-row tiles
+    (512, 384, 384, 64, 8, 1.1, "moe_experts_prefill"),    # Zipf skew, empty / hot experts, 112-row tiles
+    (100, 512, 384, 32, 4, None, "moe_experts_prefill"),   # 12.5 rows per expert: 64-row tiles
+    (3, 512, 256, 16, 4, None, "moe_experts_prefill"),     # tiny T, 16-row tiles
     (3, 512, 256, 16, 4, None, "moe_experts_decode"),      # 12 slots: 16-row tiles
     (8, 640, 384, 32, 8, None, "moe_experts_decode"),      # 64 slots: 16-row tiles, 5 k-blocks
 ])
@@ -117,10 +119,13 @@ def dsv3_mxf4(cuda_dev):
 
 
 @pytest.mark.parametrize("T,fn", [(1, "moe_experts_decode"), (8, "moe_experts_decode"),
-                                  (128, "moe_experts_prefill")])
+                                  (128, "moe_experts_prefill"), (384, "moe_experts_prefill"),
+                                  (2048, "moe_experts_prefill")])
 def test_mxf4_dsv3_sampled(moe, cuda_dev, dsv3_mxf4, T, fn):
-    """DeepSeek-V3-like layer with MXFP4 weights: T=1 / 8 take the 16-row
-    tiles, T=128 the 64-row tiles; a few tokens checked against the oracle."""
+    """DeepSeek-V3-like layer with MXFP4 weights: T=1 / 8 / 128 (<= 6 routed
+    rows per expert) take the 16-row tiles, T=384 the 64-row tiles, T=2048
+    (64 rows per expert) the 112-row tiles; a few tokens checked against the
+    oracle."""
     D = inputs.DSV3_FP8
     lay = inputs.fp8_layer(T, seed=200 + T, device=cuda_dev, weights=(None, None, None, None))
     idx, w = _route(lay, D["K"])
