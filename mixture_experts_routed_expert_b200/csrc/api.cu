@@ -10,17 +10,35 @@
 namespace moe {
 
 int num_sms() {
-    static int cache[64] = {};
+    static std::atomic<int> cache[64];   // per device ordinal (modulo 64); 0 = not read yet
     int dev = 0;
     cudaGetDevice(&dev);
-    int &c = cache[dev & 63];
+    int c = cache[dev & 63].load(std::memory_order_relaxed);
     if (c == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        c = n;
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
+            c = 148;
+        cache[dev & 63].store(c, std::memory_order_relaxed);
     }
     return c;
+}
+
+cudaError_t enable_max_dyn_smem(const void *kernel, std::atomic<int> (&done)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::atomic<int> &d = done[dev & 63];
+    if (d.load(std::memory_order_acquire)) return cudaSuccess;
+    int optin = 0;
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             optin - (int)fa.sharedSizeBytes);
+    if (e != cudaSuccess) return e;
+    d.store(1, std::memory_order_release);
+    return cudaSuccess;
 }
 
 namespace {

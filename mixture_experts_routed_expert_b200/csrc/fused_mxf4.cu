@@ -567,14 +567,9 @@ cudaError_t launch_fused_mxf4(const void *x, const void *w13, const uint8_t *w13
     while (a.stages > 2 && smem_for(a.stages) > kSmemMax) --a.stages;
     const size_t need = smem_for(a.stages);
     if (need > kSmemMax) return cudaErrorInvalidValue;
-    static size_t attr_bytes[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (attr_bytes[dev & 63] < need) {
-        err = cudaFuncSetAttribute(fused_moe_mxf4, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need);
-        if (err != cudaSuccess) return err;
-        attr_bytes[dev & 63] = need;
-    }
+    static std::atomic<int> attr_done[64];
+    err = enable_max_dyn_smem((const void *)fused_moe_mxf4, attr_done);
+    if (err != cudaSuccess) return err;
     return launch_k(fused_moe_mxf4, dim3(num_sms()), dim3(kFThreads), need, st, true, t13, t2, tx, th, a);
 }
 

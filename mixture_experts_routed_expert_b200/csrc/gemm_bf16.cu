@@ -289,16 +289,9 @@ cudaError_t launch_one(const CUtensorMap &a, const CUtensorMap &a2, const CUtens
                        cudaStream_t st) {
     using C = Cfg<GATE_UP>;
     const size_t smem = C::smem_bytes(args.E);
-    static int attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!attr_done[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_bf16<GATE_UP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)C::smem_bytes(1024));
-        if (e != cudaSuccess) return e;
-        attr_done[dev & 63] = 1;
-    }
+    static std::atomic<int> attr_done[64];
+    const cudaError_t e = enable_max_dyn_smem((const void *)grouped_gemm_bf16<GATE_UP>, attr_done);
+    if (e != cudaSuccess) return e;
     return launch_k(grouped_gemm_bf16<GATE_UP>, dim3(num_sms()), dim3(C::THREADS), smem, st, true, a,
                     a2, b, args);
 }

@@ -465,21 +465,15 @@ template <bool GATE_UP, int BN>
 cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &a2, const CUtensorMap &b,
                         const Gemm8Args &args, cudaStream_t st) {
     using C = Cfg8<GATE_UP, BN>;
-    static size_t attr_bytes[64] = {};          // per device: dynamic shared memory limit set so far
-    int dev = 0;
-    cudaGetDevice(&dev);
+    static std::atomic<int> attr_done[64];
     constexpr size_t kSmemMax = 227 * 1024;
     Gemm8Args a8 = args;
     a8.stages = C::MAX_STAGES;
     while (a8.stages > 2 && C::smem_bytes(args.E, args.KB, a8.stages) > kSmemMax) --a8.stages;
     const size_t need = C::smem_bytes(args.E, args.KB, a8.stages);
     if (need > kSmemMax) return cudaErrorInvalidValue;
-    if (attr_bytes[dev & 63] < need) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_fp8<GATE_UP, BN>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need);
-        if (e != cudaSuccess) return e;
-        attr_bytes[dev & 63] = need;
-    }
+    const cudaError_t e = enable_max_dyn_smem((const void *)grouped_gemm_fp8<GATE_UP, BN>, attr_done);
+    if (e != cudaSuccess) return e;
     return launch_k(grouped_gemm_fp8<GATE_UP, BN>, dim3(num_sms()), dim3(kThreads8), need, st, true,
                     a, a2, b, a8);
 }

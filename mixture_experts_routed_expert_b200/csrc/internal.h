@@ -2,6 +2,7 @@
 // libmoe_b200 (launchers, workspace layout, tile configuration).
 #pragma once
 
+#include <atomic>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -72,6 +73,11 @@ struct SharedSet {
 
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 int num_sms();
+// Lets `kernel` take the device's opt-in limit of dynamic shared memory (less
+// its static shared memory), once per device; `done` is the caller's
+// per-device flag array (device ordinals modulo 64).  Setting the attribute
+// is idempotent, so concurrent host threads race only on the atomic flag.
+cudaError_t enable_max_dyn_smem(const void *kernel, std::atomic<int> (&done)[64]);
 
 cudaError_t launch_permute(const int32_t *idx, int64_t n_slots, int E, int bn_g, int bn_d,
                            uint8_t *ws, const Workspace &L, cudaStream_t st);

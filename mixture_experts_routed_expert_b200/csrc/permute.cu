@@ -288,16 +288,9 @@ cudaError_t launch_pg(const void *x, const int32_t *idx, int64_t n_slots, int K,
                       int bn_g, int bn_d, uint8_t *ws, const Workspace &L, cudaStream_t st,
                       int32_t *zero = nullptr, int nzero = 0) {
     const size_t smem = sizeof(int32_t) * ((3 + kPWarps) * (size_t)E + 2);
-    static int attr_done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!attr_done[dev & 63]) {
-        cudaError_t e = cudaFuncSetAttribute(permute_gather_kernel<MODE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(sizeof(int32_t) * ((3 + kPWarps) * 1024 + 2)));
-        if (e != cudaSuccess) return e;
-        attr_done[dev & 63] = 1;
-    }
+    static std::atomic<int> attr_done[64];
+    const cudaError_t e = enable_max_dyn_smem((const void *)permute_gather_kernel<MODE>, attr_done);
+    if (e != cudaSuccess) return e;
     // about two blocks per SM for the gather; at least 128 slots per block
     // once the redundant recount of all slots becomes the larger cost
     int chunk = kPThreads;
