@@ -19,11 +19,14 @@
 //   - the MMA warp copies the scale blocks into TMEM (tcgen05.cp 32x128b,
 //     all four lane quarters) and issues four MMAs of K = 32 per k-block,
 //     each selecting its scale byte.
-// Tiles and epilogues as in the E4M3 kernel.  Warp roles: warp 0 TMA
-// producer, warps 1 and 10 MMA issue (warp 1 also allocates TMEM), warps 2-9
-// epilogue from double-buffered TMEM accumulators.  With a few routed rows per
-// tile an MMA instruction does little tensor work, and two issuing warps keep
-// the tensor cores fed where one could not: gate_up issues gate and up from
+// Tiles as in the E4M3 kernel, of 16, 64 or 112 routed rows (the MMA's N);
+// the epilogue walks a tile in chunks of 32 accumulator columns.  Warp roles:
+// warps 0 and 11 TMA producers (gate_up: gate weights and the activation
+// tile with its scales / up weights; down: weights / activations and scales),
+// warps 1 and 10 MMA issue (warp 1 also allocates TMEM), warps 2-9 epilogue
+// from double-buffered TMEM accumulators.  With a few routed rows per tile an
+// MMA instruction does little tensor work, and two issuing warps keep the
+// tensor cores fed where one could not: gate_up issues gate and up from
 // separate warps, down the two k-blocks of each stage into two partial
 // accumulators that the epilogue adds.
 //   S4 (gate_up): h = bf16(SiLU(g) * u), quantised per 128 features (the
