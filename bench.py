@@ -317,8 +317,11 @@ def run_ours(args):
 
     # ---- end to end through the C ABI with host buffers -------------------
     # The step's inputs (x, top-k ids, top-k weights) sit in one pinned host
-    # buffer and go over in one copy; the step (copy in, decode, copy out) is
-    # captured once and replayed, as a serving loop would.
+    # buffer, mapped into the device's address space, and moe_stage_inputs
+    # moves them to the device with one kernel; the decode kernels write the
+    # output straight into mapped pinned host memory (the C ABI takes any
+    # device-accessible pointer).  The step is captured once and replayed, as
+    # a serving loop would.
     def packed(tensors):
         offs, o = [], 0
         for t_ in tensors:
@@ -327,31 +330,45 @@ def run_ours(args):
         return offs, o
     ins = [lay1.x, lay1.idx, lay1.w]
     offs, nbytes = packed(ins)
-    hbuf = torch.zeros(nbytes, dtype=torch.uint8).pin_memory()
     dbuf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     views_d = []
     for t_, o in zip(ins, offs):
         nb = t_.numel() * t_.element_size()
-        hbuf[o:o + nb].copy_(t_.cpu().contiguous().view(-1).view(torch.uint8))
         views_d.append(dbuf[o:o + nb].view(t_.dtype).view(t_.shape))
     xd, idd, wd = views_d
-    # The output goes straight into mapped pinned host memory (the kernels
-    # write it over the bus; the C ABI takes any device-accessible pointer).
     out_bytes = out1.numel() * 2
+    in_map = mapped_host_buffer(nbytes)
     mapped = mapped_host_buffer(out_bytes)
-    if mapped is not None:
+    host_mem = []
+    if in_map is not None and mapped is not None:
+        h_in, d_in = in_map
         h_out, d_out = mapped
+        host_mem = [h_in, h_out]
+        for t_, o in zip(ins, offs):
+            b = t_.cpu().contiguous().view(-1).view(torch.uint8).numpy().tobytes()
+            ctypes.memmove(h_in + o, b, len(b))
         C = ctypes.c_void_p
 
         def e2e_call():
-            dbuf.copy_(hbuf, non_blocking=True)
+            st_ = C(torch.cuda.current_stream().cuda_stream)
+            rc = moe.lib.moe_stage_inputs(C(d_in), C(dbuf.data_ptr()), nbytes, st_)
+            assert rc == 0, rc
             rc = moe.lib.moe_experts_decode(
                 C(xd.data_ptr()), C(lay1.gate_up.data_ptr()), C(lay1.down.data_ptr()),
                 C(idd.data_ptr()), C(wd.data_ptr()), K, 1, H, F, E, 0, None, None, C(d_out),
-                C(ws1.data_ptr()), ws1.numel(), C(torch.cuda.current_stream().cuda_stream))
+                C(ws1.data_ptr()), ws1.numel(), st_)
             assert rc == 0, rc
-        e2e_how = "one copy of the pinned inputs, decode writing out into mapped pinned host memory"
+        e2e_how = ("inputs in mapped pinned host memory moved by moe_stage_inputs (one kernel), "
+                   "decode writing out into mapped pinned host memory")
     else:
+        for hm in (in_map, mapped):
+            if hm is not None:
+                free_mapped_host_buffer(hm[0])
+        mapped = None
+        hbuf = torch.zeros(nbytes, dtype=torch.uint8).pin_memory()
+        for t_, o in zip(ins, offs):
+            nb = t_.numel() * t_.element_size()
+            hbuf[o:o + nb].copy_(t_.cpu().contiguous().view(-1).view(torch.uint8))
         oh = torch.empty_like(out1, device="cpu").pin_memory()
 
         def e2e_call():
@@ -373,8 +390,10 @@ def run_ours(args):
         host_out = np.frombuffer(ctypes.string_at(h_out, out_bytes), dtype=np.uint16)
         dev_out = out1.view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
         assert np.array_equal(host_out, dev_out), "replayed step did not write the output"
-        free_mapped_host_buffer(h_out)
     del e2e_graph
+    torch.cuda.synchronize()
+    for hm in host_mem:
+        free_mapped_host_buffer(hm)
 
     # ---- breakdown: other decode sizes, eager decode, OCR-2 prefill ---------
     breakdown = {}

@@ -243,6 +243,24 @@ MOE_API moe_status_t moe_experts_decode_static(const void *hidden_states, const 
                                        const void *down_scale, void *out, void *stream);
 
 /*
+ * Host-input staging for a step (no operation of the method: plumbing for
+ * callers whose inputs arrive in host memory).  Copies `bytes` bytes from
+ * `src` to the device memory `dst` with one kernel on `stream`.  `src` is
+ * memory the GPU can read, typically pinned host memory allocated mapped
+ * (cudaHostAllocMapped; pass its device pointer) that holds a step's hidden
+ * states, top-k ids and top-k weights packed in one buffer.  Every load of
+ * src bypasses the caches (ld.global.cv), so host writes made before the call
+ * is enqueued are seen; the host must not modify src until the stream has
+ * passed the call.  For the few KB of a decode step's inputs the kernel ends
+ * sooner than a copy-engine transfer (cudaMemcpyAsync).
+ *  - bytes: a multiple of 16, at most 1 GiB; src and dst 16-byte aligned and
+ *    not overlapping; both buffers stay the caller's.
+ *  - Returns MOE_OK (bytes == 0 is a no-op), MOE_ERR_INVALID_ARG (null or
+ *    misaligned pointer, bad size) or MOE_ERR_CUDA.
+ */
+MOE_API moe_status_t moe_stage_inputs(const void *src, void *dst, size_t bytes, void *stream);
+
+/*
  * Group-aware sigmoid top-k routing (layer table:
  * moe_topk_sigmoid_routing_layer, num_groups=8, topk_group=4,
  * routed_scaling_factor=2.5 for DeepSeek-V3).

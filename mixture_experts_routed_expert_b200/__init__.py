@@ -27,7 +27,7 @@ EXPORTS = ("moe_abi_version", "moe_status_string", "moe_experts_workspace_size",
            "moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
            "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
            "moe_experts_shared_workspace_size", "moe_experts_with_shared",
-           "moe_experts_decode_fused")
+           "moe_experts_decode_fused", "moe_stage_inputs")
 
 
 def _load():
@@ -52,9 +52,10 @@ def _load():
     L.moe_experts_shared_workspace_size.argtypes = [I, I, I, I, I, I, I]
     L.moe_experts_with_shared.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P,
                                           P, P, P, P, I, P, P, P, Z, P]
+    L.moe_stage_inputs.argtypes = [P, P, Z, P]
     for n in ("moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
               "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
-              "moe_experts_with_shared", "moe_experts_decode_fused"):
+              "moe_experts_with_shared", "moe_experts_decode_fused", "moe_stage_inputs"):
         getattr(L, n).restype = I
     return L
 
@@ -225,6 +226,16 @@ def moe_experts_decode_static(hidden_states, gate_up_proj, down_proj, top_k_inde
                                        _ptr(down_scale), _ptr(out), _stream(stream))
     _check(rc, "moe_experts_decode_static")
     return out
+
+
+def moe_stage_inputs(src_ptr, dst, nbytes=None, stream=None):
+    """Copy `nbytes` (default: all of dst) from the device-readable address
+    `src_ptr` (an int, e.g. the device pointer of mapped pinned host memory)
+    into the device tensor `dst` with one kernel on the stream."""
+    nbytes = dst.numel() * dst.element_size() if nbytes is None else nbytes
+    rc = lib.moe_stage_inputs(ctypes.c_void_p(src_ptr), _ptr(dst), nbytes, _stream(stream))
+    _check(rc, "moe_stage_inputs")
+    return dst
 
 
 def moe_route_sigmoid_grouped(logits, bias, num_groups, topk_group, top_k, routed_scaling_factor,

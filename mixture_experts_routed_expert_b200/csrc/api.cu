@@ -437,4 +437,11 @@ moe_status_t moe_debug_permute(const int32_t *top_k_index, int T, int K, int E, 
     return from_cuda(e);
 }
 
+moe_status_t moe_stage_inputs(const void *src, void *dst, size_t bytes, void *stream) {
+    if (bytes == 0) return MOE_OK;
+    if (!src || !dst || (bytes & 15) || !aligned16(src) || !aligned16(dst) || bytes > ((size_t)1 << 30))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_stage_copy(src, dst, bytes, (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -126,6 +126,9 @@ cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *d
                                const void *residual = nullptr);
 cudaError_t launch_quantize(const void *x, int64_t rows, int cols, void *xq, float *scale,
                             cudaStream_t st);
+// One kernel copying bytes (a multiple of 16) from src to dst, src read with
+// cache-volatile loads (it may be mapped pinned host memory).
+cudaError_t launch_stage_copy(const void *src, void *dst, size_t bytes, cudaStream_t st);
 cudaError_t launch_route(const float *logits, const float *bias, int64_t T, int E, int num_groups,
                          int topk_group, int top_k, float scale, int32_t *idx, float *w,
                          int32_t *offsets, cudaStream_t st);

@@ -66,6 +66,11 @@ def test_host_validation_without_gpu(mod):
     # quantiser limits
     assert L.quantize_fp8_block128(p, 4, 100, p, p, N) == 1
     assert L.quantize_fp8_block128(p, 0, 128, p, p, N) == 0
+    # input staging: sizes in 16-byte units, aligned pointers
+    assert L.moe_stage_inputs(N, N, 0, N) == 0
+    assert L.moe_stage_inputs(p, p, 24, N) == 1
+    assert L.moe_stage_inputs(q, p, 32, N) == 1
+    assert L.moe_stage_inputs(p, N, 32, N) == 1
 
 
 def test_shared_entry_host_checks(mod):
