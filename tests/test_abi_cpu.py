@@ -120,3 +120,44 @@ def test_mxfp4_host_checks(mod):
     f = L.moe_experts_with_shared
     assert f(p, p, p, p, p, 8, 4, 7168, 2048, 256, W, p, p, p, p, N, N, 1, N, p, p, big, N) == 2
     assert L.moe_experts_decode_static(p, p, p, p, p, 6, 1, 1280, 896, 64, W, p, p, p, N) == 2
+
+
+def test_binding_argument_checks(mod):
+    """The Python binding rejects wrong shapes, dtypes and devices before any
+    C call, and maps weight dtypes (and weight_format) to the C weight type."""
+    import torch
+    T, H, F, E, K = 4, 256, 128, 8, 2
+    x = torch.zeros(T, H, dtype=torch.bfloat16)
+    gu = torch.zeros(E, 2 * F, H, dtype=torch.bfloat16)
+    dn = torch.zeros(E, H, F, dtype=torch.bfloat16)
+    idx = torch.zeros(T, K, dtype=torch.int32)
+    w = torch.zeros(T, K, dtype=torch.float32)
+    fwd = mod.moe_experts_prefill
+    with pytest.raises(ValueError, match="shape mismatch"):
+        fwd(x[:, :128], gu, dn, idx, w, K)
+    with pytest.raises(ValueError, match="shape mismatch"):
+        fwd(x, gu, dn[:, :, :64], idx, w, K)
+    with pytest.raises(ValueError, match="top_k"):
+        fwd(x, gu, dn, idx[:, :1], w, K)
+    with pytest.raises(TypeError, match="int32"):
+        fwd(x, gu, dn, idx.long(), w, K)
+    with pytest.raises(TypeError, match="bf16"):
+        fwd(x.float(), gu, dn, idx, w, K)
+    with pytest.raises(ValueError, match="CUDA"):       # host tensors never reach the library
+        fwd(x, gu, dn, idx, w, K)
+    # packed MXFP4 shapes: gate_up [E][2F][H/2], down [E][H][F/2]
+    gu4 = torch.zeros(E, 2 * F, H // 2, dtype=torch.uint8)
+    dn4 = torch.zeros(E, H, F // 2, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        fwd(x, gu4, dn4, idx, w, K, weight_format="mxfp4")
+    with pytest.raises(ValueError, match="shape mismatch"):
+        fwd(x, gu4, dn4, idx, w, K)                     # read as E4M3: H/2 columns
+    wt = mod._wtype
+    assert wt(gu) == mod.MOE_W_BF16
+    assert wt(gu4) == mod.MOE_W_FP8_E4M3
+    assert wt(gu4.view(torch.float8_e4m3fn)) == mod.MOE_W_FP8_E4M3
+    assert wt(gu4, "mxfp4") == mod.MOE_W_MXFP4
+    with pytest.raises(TypeError):
+        wt(gu, "mxfp4")
+    with pytest.raises(TypeError):
+        wt(gu.float())
