@@ -223,15 +223,22 @@ MOE_API moe_status_t moe_experts_with_shared(
  * the code they load no allocator.  The pages have no counterpart of this
  * entry point; it exists for those callers only.
  *
- * Same arguments, layouts and results as moe_experts_decode, minus the
- * workspace.  Its scratch memory is a fixed 1 MiB array inside the library
- * that every GPU which loads the library holds until the process exits.
- * The library itself allocates nothing and calls no allocating routine.
- *  - Sizes whose decode scratch (moe_experts_workspace_size(..., 1)) exceeds
- *    1 MiB, and calls outside the decode range (T > 16 or T*K > 64), return
- *    MOE_ERR_WORKSPACE; e4m3 and MXFP4 weights return MOE_ERR_UNSUPPORTED.
- *  - The first call on a device looks up the array's device address with
- *    that device current; make that first call before any stream capture.
+ * Same arguments and layouts as moe_experts_decode, minus the workspace;
+ * results equal moe_experts_decode's within the parity tolerance (relative
+ * L2 error <= 5e-3), not always bit for bit: this entry always runs the
+ * gather-GEMV decode kernels, which serve up to 64 slots (T*K), while
+ * moe_experts_decode hands calls above 16 slots to the grouped GEMMs.  Its
+ * scratch memory is a fixed 1 MiB array inside the library that every GPU
+ * which loads the library holds until the process exits; 1 MiB is above the
+ * largest decode scratch (64 slots x 2048 features of bf16 h).  The library
+ * itself allocates nothing and calls no allocating routine.
+ *  - bf16 weights only: e4m3 and MXFP4 weights return MOE_ERR_UNSUPPORTED;
+ *    calls outside the decode range (T > 16, T*K > 64, H or F > 2048)
+ *    return MOE_ERR_WORKSPACE.
+ *  - Every call looks up the array's device address in the current context
+ *    (after a cudaDeviceReset the next call finds the new one).  The first
+ *    call in a context loads the library's device code there: make it before
+ *    any stream capture.
  *  - All calls share the one array, which keeps the last call's contents:
  *    calls that may overlap on the GPU (other streams, or other host threads
  *    without ordering) race on it and must be serialised by the caller.

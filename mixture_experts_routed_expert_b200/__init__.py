@@ -7,7 +7,11 @@ name; all arithmetic runs in the library's CUDA kernels.  torch is used for
 device memory (outputs, workspaces) and streams only.
 
 The library must be built (``python mixture_experts_routed_expert_b200/build.py``
-or ``__graft_entry__.build()``); importing this package without it raises.
+or ``__graft_entry__.build()``).  It is loaded on first use -- the first
+call of an entry point or the first access to ``lib`` -- so that the input
+recipe (``mixture_experts_routed_expert_b200.inputs``) imports without it;
+every entry point raises ImportError when it is missing.  There is no CPU
+fallback.
 """
 import ctypes
 import os
@@ -60,7 +64,22 @@ def _load():
     return L
 
 
-lib = _load()
+_LIB = None
+
+
+def _lib():
+    """The loaded library (loaded on the first call; raises ImportError when
+    libmoe_b200.so is not built)."""
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _lib()
+    raise AttributeError("module %r has no attribute %r" % (__name__, name))
 
 
 class MoEError(RuntimeError):
@@ -97,12 +116,15 @@ def _wtype(gate_up_proj, weight_format=None):
 
 
 def moe_experts_workspace_size(T, H, F, E, K, wtype=MOE_W_BF16, decode=False):
-    return int(lib.moe_experts_workspace_size(T, H, F, E, K, wtype, int(bool(decode))))
+    return int(_lib().moe_experts_workspace_size(T, H, F, E, K, wtype, int(bool(decode))))
 
 
-def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
-             gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None,
-             weight_format=None):
+def _check_forward_args(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
+                        top_k, gate_up_scale=None, down_scale=None, out=None, weight_format=None):
+    """Shape, dtype and device checks of the forward entry points, made before
+    any C call (the library sees only raw pointers and cannot detect a host
+    tensor, a non-contiguous view or a wrong integer width).  Returns
+    (T, H, F, E, weight type)."""
     T, H = hidden_states.shape
     E, F2, H2 = gate_up_proj.shape
     packed = weight_format == "mxfp4"          # two codes per byte along the reduction
@@ -117,18 +139,29 @@ def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_we
         raise TypeError("top_k_index must be int32 and top_k_weights float32")
     if hidden_states.dtype != torch.bfloat16:
         raise TypeError("hidden_states must be bf16")
+    if out is not None and (tuple(out.shape) != (T, H) or out.dtype != torch.bfloat16):
+        raise ValueError("out must be [T, H] bf16")
     for t in (hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, gate_up_scale,
-              down_scale):
+              down_scale, out):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("all tensors must be contiguous CUDA tensors")
-    wt = _wtype(gate_up_proj, weight_format)
+    return T, H, F2 // 2, E, _wtype(gate_up_proj, weight_format)
+
+
+def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
+             gate_up_scale=None, down_scale=None, out=None, workspace=None, stream=None,
+             weight_format=None):
+    T, H, F, E, wt = _check_forward_args(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                         top_k_weights, top_k, gate_up_scale, down_scale, out,
+                                         weight_format)
+    F2 = 2 * F
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
     decode = name in ("moe_experts_decode", "moe_experts_decode_fused")
     need = moe_experts_workspace_size(T, H, F2 // 2, E, top_k, wt, decode)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=hidden_states.device)
-    rc = getattr(lib, name)(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
+    rc = getattr(_lib(), name)(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
                             _ptr(top_k_index), _ptr(top_k_weights), top_k, T, H, F2 // 2, E, wt,
                             _ptr(gate_up_scale), _ptr(down_scale), _ptr(out), _ptr(workspace),
                             workspace.numel() * workspace.element_size(), _stream(stream))
@@ -157,7 +190,7 @@ def moe_experts_decode(hidden_states, gate_up_proj, down_proj, top_k_index, top_
 
 
 def moe_experts_shared_workspace_size(T, H, F, E, K, S, wtype=MOE_W_BF16):
-    return int(lib.moe_experts_shared_workspace_size(T, H, F, E, K, S, wtype))
+    return int(_lib().moe_experts_shared_workspace_size(T, H, F, E, K, S, wtype))
 
 
 def moe_experts_with_shared(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
@@ -191,7 +224,7 @@ def moe_experts_with_shared(hidden_states, gate_up_proj, down_proj, top_k_index,
     need = moe_experts_shared_workspace_size(T, H, F, E, top_k, S, wt)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=hidden_states.device)
-    rc = lib.moe_experts_with_shared(
+    rc = _lib().moe_experts_with_shared(
         _ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj), _ptr(top_k_index),
         _ptr(top_k_weights), top_k, T, H, F, E, wt, _ptr(gate_up_scale), _ptr(down_scale),
         _ptr(shared_gate_up_proj), _ptr(shared_down_proj), _ptr(shared_gate_up_scale),
@@ -215,15 +248,16 @@ def moe_experts_decode_static(hidden_states, gate_up_proj, down_proj, top_k_inde
                               top_k, gate_up_scale=None, down_scale=None, out=None, stream=None):
     """Decode form without a workspace: scratch comes from a fixed 1 MiB array
     inside the library (for callers that cannot allocate device memory; calls
-    that overlap on the GPU race on that array)."""
-    T, H = hidden_states.shape
-    E, F2, _ = gate_up_proj.shape
+    that overlap on the GPU race on that array).  The same argument checks as
+    moe_experts_decode run first."""
+    T, H, F, E, wt = _check_forward_args(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                         top_k_weights, top_k, gate_up_scale, down_scale, out)
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
-    rc = lib.moe_experts_decode_static(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
-                                       _ptr(top_k_index), _ptr(top_k_weights), top_k, T, H, F2 // 2,
-                                       E, _wtype(gate_up_proj), _ptr(gate_up_scale),
-                                       _ptr(down_scale), _ptr(out), _stream(stream))
+    rc = _lib().moe_experts_decode_static(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
+                                          _ptr(top_k_index), _ptr(top_k_weights), top_k, T, H, F,
+                                          E, wt, _ptr(gate_up_scale), _ptr(down_scale), _ptr(out),
+                                          _stream(stream))
     _check(rc, "moe_experts_decode_static")
     return out
 
@@ -233,7 +267,7 @@ def moe_stage_inputs(src_ptr, dst, nbytes=None, stream=None):
     `src_ptr` (an int, e.g. the device pointer of mapped pinned host memory)
     into the device tensor `dst` with one kernel on the stream."""
     nbytes = dst.numel() * dst.element_size() if nbytes is None else nbytes
-    rc = lib.moe_stage_inputs(ctypes.c_void_p(src_ptr), _ptr(dst), nbytes, _stream(stream))
+    rc = _lib().moe_stage_inputs(ctypes.c_void_p(src_ptr), _ptr(dst), nbytes, _stream(stream))
     _check(rc, "moe_stage_inputs")
     return dst
 
@@ -250,7 +284,7 @@ def moe_route_sigmoid_grouped(logits, bias, num_groups, topk_group, top_k, route
         top_k_weights = torch.empty(T, top_k, dtype=torch.float32, device=dev)
     if want_offsets and expert_offsets is None:
         expert_offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
-    rc = lib.moe_route_sigmoid_grouped(_ptr(logits), _ptr(bias), T, E, num_groups, topk_group,
+    rc = _lib().moe_route_sigmoid_grouped(_ptr(logits), _ptr(bias), T, E, num_groups, topk_group,
                                        top_k, float(routed_scaling_factor), _ptr(top_k_index),
                                        _ptr(top_k_weights), _ptr(expert_offsets), _stream(stream))
     _check(rc, "moe_route_sigmoid_grouped")
@@ -266,7 +300,7 @@ def quantize_fp8_block128(x, xq=None, scale=None, stream=None):
         xq = torch.empty(rows, cols, dtype=torch.uint8, device=x.device)
     if scale is None:
         scale = torch.empty(rows, cols // 128, dtype=torch.float32, device=x.device)
-    rc = lib.quantize_fp8_block128(_ptr(x), rows, cols, _ptr(xq), _ptr(scale), _stream(stream))
+    rc = _lib().quantize_fp8_block128(_ptr(x), rows, cols, _ptr(xq), _ptr(scale), _stream(stream))
     _check(rc, "quantize_fp8_block128")
     return xq, scale
 
@@ -282,7 +316,7 @@ def moe_debug_permute(top_k_index, E, workspace=None, stream=None):
     need = moe_experts_workspace_size(T, 128, 128, E, K, MOE_W_BF16, False)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    rc = lib.moe_debug_permute(_ptr(top_k_index), T, K, E, _ptr(counts), _ptr(offsets), _ptr(perm),
+    rc = _lib().moe_debug_permute(_ptr(top_k_index), T, K, E, _ptr(counts), _ptr(offsets), _ptr(perm),
                                _ptr(inv), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "moe_debug_permute")
     return counts, offsets, perm[:T * K], inv[:T * K]

@@ -12,14 +12,14 @@
 // The array is a file-scope __device__ object, so every GPU that loads the
 // library holds kStaticScratchBytes of it until the process exits.  Host code
 // must not use the array's name as a device address: on the host the name
-// only denotes a stand-in object.  The device address is obtained once per
-// device with cudaGetSymbolAddress, with that device current, on the first
-// call on that device (that first call should therefore come before any
-// stream capture).  All calls share the one array and it keeps whatever the
-// last call left there: calls that may overlap on the GPU (different streams,
-// or different host threads without ordering) race on it.
-#include <mutex>
-
+// only denotes a stand-in object.  Every call looks up the device address
+// with cudaGetSymbolAddress in the caller's current context (a host-side
+// query: no stream work, no allocation), so the address stays right after a
+// cudaDeviceReset or when another context is current.  The first call in a
+// context also loads the library's module there, so it should come before
+// any stream capture.  All calls share the one array and it keeps whatever
+// the last call left there: calls that may overlap on the GPU (different
+// streams, or different host threads without ordering) race on it.
 #include "internal.h"
 
 namespace moe {
@@ -30,23 +30,18 @@ constexpr size_t kStaticScratchBytes = 1u << 20;   // 1 MiB
 
 __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mutex;
-void *g_scratch_addr[64] = {};
+// The largest decode scratch (T*K <= kDecodeMaxSlots slots of h, F <= 2048
+// features, plus the status words) fits the array, so every size the decode
+// kernels accept is served.
+static_assert(256 + (size_t)kDecodeMaxSlots * 2048 * 2 <= kStaticScratchBytes,
+              "static decode scratch smaller than the largest decode workspace");
 
-// Device address of g_decode_scratch on the current device (looked up once).
+// Device address of g_decode_scratch in the current context.
 cudaError_t scratch_address(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -65,8 +60,8 @@ extern "C" MOE_API moe_status_t moe_experts_decode_static(
                                       top_k_weights, top_k, T, H, F, E, wt, gate_up_scale,
                                       down_scale, out);
     if (s != MOE_OK || T == 0) return s;
-    if (!decode_path_fits(T, top_k, H, F)) return MOE_ERR_WORKSPACE;
     if (wt != MOE_W_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!decode_path_fits(T, top_k, H, F)) return MOE_ERR_WORKSPACE;
     const DecodeWorkspace L = decode_workspace(T, H, F, E, top_k, wt);
     if (L.total > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
     void *scratch = nullptr;

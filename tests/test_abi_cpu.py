@@ -17,6 +17,23 @@ def mod():
     return m
 
 
+def test_input_recipe_loads_no_library():
+    """The seeded input recipe imports without loading libmoe_b200.so (the
+    oracle-only reference arm uses it), while the entry points load it."""
+    import subprocess
+    import sys
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from mixture_experts_routed_expert_b200 import inputs\n"
+            "inputs.ocr2_layer(2, seed=0, H=128, F=128, E=4, K=2)\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "assert 'libmoe_b200' not in maps, 'library mapped by the input recipe'\n"
+            "import mixture_experts_routed_expert_b200 as m\n"
+            "m.lib.moe_abi_version()\n"
+            "assert 'libmoe_b200' in open('/proc/self/maps').read()\n" % ROOT)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+
+
 def test_exports_match_header(mod):
     decl = set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(", open(HEADER).read()))
     assert decl == set(mod.EXPORTS)
@@ -152,6 +169,18 @@ def test_binding_argument_checks(mod):
         fwd(x, gu4, dn4, idx, w, K, weight_format="mxfp4")
     with pytest.raises(ValueError, match="shape mismatch"):
         fwd(x, gu4, dn4, idx, w, K)                     # read as E4M3: H/2 columns
+    # the static-scratch decode entry runs the same checks before its C call
+    st = mod.moe_experts_decode_static
+    with pytest.raises(ValueError, match="shape mismatch"):
+        st(x, gu, dn[:, :, :64], idx, w, K)
+    with pytest.raises(TypeError, match="int32"):
+        st(x, gu, dn, idx.long(), w, K)
+    with pytest.raises(TypeError, match="bf16"):
+        st(x.float(), gu, dn, idx, w, K)
+    with pytest.raises(ValueError, match="CUDA"):
+        st(x, gu, dn, idx, w, K)
+    with pytest.raises(ValueError, match="out must be"):
+        st(x, gu, dn, idx, w, K, out=torch.zeros(T, H + 128, dtype=torch.bfloat16))
     wt = mod._wtype
     assert wt(gu) == mod.MOE_W_BF16
     assert wt(gu4) == mod.MOE_W_FP8_E4M3

@@ -7,12 +7,11 @@ tiles for few routed rows per expert, 112-row tiles for many, 64-row tiles
 between), and sampled tokens of the
 DeepSeek-V3-like layer (H=7168, F=2048, E=256, K=8) with MXFP4 weights; the
 one-kernel decode form (moe_experts_decode_fused) on the same checks."""
-import numpy as np
 import pytest
 import torch
 
 import oracle
-from _helpers import assert_matches_oracle
+from _helpers import assert_matches_oracle, grouped_tile_heights, parity_sample
 from mixture_experts_routed_expert_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -125,36 +124,17 @@ def dsv3_mxf4(cuda_dev):
 def test_mxf4_dsv3_sampled(moe, cuda_dev, dsv3_mxf4, T, fn):
     """DeepSeek-V3-like layer with MXFP4 weights: T=1 / 8 / 128 (<= 6 routed
     rows per expert) take the 16-row tiles, T=384 the 64-row tiles, T=2048
-    (64 rows per expert) the 112-row tiles; a few tokens checked against the
-    oracle."""
+    (64 rows per expert) the 112-row tiles; sampled tokens (the hottest
+    expert's last row tile, the rarest expert's tokens, >= 16 in all)
+    checked against the oracle."""
     D = inputs.DSV3_FP8
     lay = inputs.fp8_layer(T, seed=200 + T, device=cuda_dev, weights=(None, None, None, None))
     idx, w = _route(lay, D["K"])
     out = _run(moe, lay.x, dsv3_mxf4, idx, w, cuda_dev, fn)
-    tokens = sorted({0, T // 2, T - 1})
+    tokens = parity_sample(idx.numpy(), D["E"], grouped_tile_heights(T, D["K"], D["E"], "mxfp4"),
+                           seed=T)
     ref = _oracle(lay.x, dsv3_mxf4, idx, w, D["E"], tokens=tokens)
     assert_matches_oracle(out[tokens], ref, "mxf4 dsv3 T=%d" % T)
-
-
-@pytest.mark.parametrize("T", [64, 2048, 8192])
-def test_mxf4_dsv3_zipf_sweep_sampled(moe, cuda_dev, dsv3_mxf4, T):
-    """Zipf(1.1) expert popularity over the 256 experts with MXFP4 weights:
-    at T >= 2048 the hot experts take many 112-row tiles and some experts
-    none; tokens routed to the hottest expert and the first and last token
-    checked against the oracle."""
-    D = inputs.DSV3_FP8
-    lay = inputs.fp8_layer(T, seed=7 * T, device=cuda_dev, zipf=1.1,
-                           weights=(None, None, None, None))
-    idx, w = _route(lay, D["K"])
-    counts = np.bincount(idx.numpy().reshape(-1), minlength=D["E"])
-    if T >= 2048:
-        assert counts.max() > 112 and (counts == 0).any()
-    out = _run(moe, lay.x, dsv3_mxf4, idx, w, cuda_dev)
-    hot = int(counts.argmax())
-    rows = torch.nonzero((idx == hot).any(dim=1)).reshape(-1)
-    tokens = sorted({int(r) for r in rows[:2]} | {0, T - 1})
-    ref = _oracle(lay.x, dsv3_mxf4, idx, w, D["E"], tokens=tokens)
-    assert_matches_oracle(out[tokens], ref, "mxf4 dsv3 zipf T=%d" % T)
 
 
 def test_mxf4_zero_tokens_and_zero_weights(moe, cuda_dev):

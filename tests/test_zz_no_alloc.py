@@ -55,6 +55,9 @@ def test_decode_static_rejects_oversize(cuda_dev):
     import mixture_experts_routed_expert_b200 as moe
     lib = moe.lib
     p = ctypes.c_void_p(256)
-    # T*K beyond the decode range, and a scratch need above the 1 MiB array
+    # outside the decode range: T*K > 64, and F > 2048 (every size inside the
+    # range fits the 1 MiB array, which the library checks at compile time)
     assert lib.moe_experts_decode_static(p, p, p, p, p, 8, 16, 1280, 896, 64, 0, None, None, p, None) == 3
     assert lib.moe_experts_decode_static(p, p, p, p, p, 16, 4, 1280, 16384, 64, 0, None, None, p, None) == 3
+    # quantised weights are not served, whatever the sizes
+    assert lib.moe_experts_decode_static(p, p, p, p, p, 8, 16, 1280, 896, 64, 1, p, p, p, None) == 2
