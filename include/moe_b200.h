@@ -35,6 +35,13 @@
  *  - Expert ids outside [0, E) contribute nothing to the output.
  *  - Calls on the same stream may reuse the same workspace; calls that may
  *    overlap (different streams) need separate workspaces.
+ *  - Every workspace begins with an 8 KiB header: the int32 device status
+ *    word at offset 0 (bits set by a kernel whose bounded wait expired) and
+ *    the arrival counters of the fused bf16 decode kernel.  The header must
+ *    be zero before a workspace's first use (allocate it zero-filled, or call
+ *    moe_workspace_init once); every call that completes leaves it zero
+ *    again.  After moe_workspace_status reports MOE_ERR_TIMEOUT, clear it
+ *    (moe_workspace_status(..., clear = 1) does) before the next call.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -58,7 +65,8 @@ typedef enum {
     MOE_ERR_UNSUPPORTED = 2,   /* shape or mode outside what is implemented */
     MOE_ERR_WORKSPACE = 3,     /* workspace missing or too small            */
     MOE_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed       */
-    MOE_ERR_TIMEOUT = 5        /* reserved: a bounded device wait expired   */
+    MOE_ERR_TIMEOUT = 5        /* a bounded device wait of an earlier call
+                                  expired (moe_workspace_status)             */
 } moe_status_t;
 
 typedef enum {
@@ -112,7 +120,9 @@ MOE_API size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe
  *                            pointer, e.g. mapped pinned host memory: the
  *                            kernels store it directly)
  *   workspace      device scratch of >= moe_experts_workspace_size(..., 0)
- *                  bytes, 256-byte aligned; contents need no initialisation
+ *                  bytes, 256-byte aligned; its 8 KiB header zero before
+ *                  first use (see the conventions above), the rest needs no
+ *                  initialisation
  *
  * bf16 path: h = bf16(SiLU(g) * u) is stored in bf16 between the GEMMs;
  * fp32 accumulation everywhere; the K contributions of a token are summed in
@@ -136,9 +146,15 @@ MOE_API moe_status_t moe_experts_prefill(const void *hidden_states, const void *
  * Routed-experts forward, decode form: a fused gather-GEMV for a few tokens
  * (model card op "deepseek_ocr2_moe_experts_decode", n_tokens about 1-4).
  * Same arguments, layouts and results as moe_experts_prefill, workspace from
- * moe_experts_workspace_size(..., 1).  Tuned for T * K <= 64 (bf16: two
- * gather-GEMV kernels; E4M3: the grouped GEMMs with 16-row activation
- * tiles); larger calls are served by the prefill kernels (same results).
+ * moe_experts_workspace_size(..., 1).  Tuned for T * K <= 64.  bf16 weights
+ * with T <= 16 and H, F <= 2048: one kernel launch (expert dedup, gate/up
+ * GEMV with SiLU*up, down GEMV, router-weight scale and the fixed-order
+ * top-K combine), launched as a programmatic dependent of the previous
+ * kernel on the stream (it reads no input before that kernel has finished);
+ * it counts on the workspace header being zero (see the conventions above).
+ * E4M3 and MXFP4 weights: the grouped GEMMs with 16-row activation tiles.
+ * Larger calls are served by the prefill kernels (same results within the
+ * parity tolerance).
  */
 MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_proj,
                                 const void *down_proj, const int32_t *top_k_index,
@@ -248,6 +264,47 @@ MOE_API moe_status_t moe_experts_decode_static(const void *hidden_states, const 
                                        const float *top_k_weights, int top_k, int T, int H, int F,
                                        int E, moe_wtype_t wt, const void *gate_up_scale,
                                        const void *down_scale, void *out, void *stream);
+
+/*
+ * Zeroes the 8 KiB header of a workspace (status word and counters),
+ * asynchronously on `stream`; needed once before a workspace's first use
+ * unless it was allocated zero-filled.  No allocation.
+ *   workspace_bytes >= 8192; workspace 256-byte aligned.
+ * Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_CUDA.
+ */
+MOE_API moe_status_t moe_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Device status of the calls that used `workspace`: waits for `stream`
+ * (the one entry point that synchronises the host), reads the status word
+ * and returns MOE_ERR_TIMEOUT when a bounded device wait of one of those
+ * calls expired (that call's outputs are undefined), MOE_OK otherwise.
+ * clear != 0 then zeroes the workspace header (status word and counters),
+ * so that the workspace can be used again.  Grouped-GEMM (prefill-path)
+ * calls restart the status word themselves; the fused decode kernel only
+ * ever sets bits in it.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT, MOE_ERR_INVALID_ARG or MOE_ERR_CUDA.
+ */
+MOE_API moe_status_t moe_workspace_status(void *workspace, int clear, void *stream);
+
+/*
+ * Test-only form of moe_experts_decode for the fused bf16 decode kernel that
+ * exercises its timeout path: CTA 0 never issues the weight copies of its
+ * work chunk number `withhold_chunk` (0 = its first), so its bounded wait
+ * for them expires (after about 2 s of SM clock cycles); the kernel then
+ * sets MOE_ERR_TIMEOUT's status bit, drains its own copies and returns
+ * without faulting.  The outputs of such a call are undefined.  Same
+ * arguments as moe_experts_decode (bf16 weights, fused decode sizes only:
+ * MOE_ERR_UNSUPPORTED otherwise).  Not part of the method (the pages have no
+ * counterpart); it exists so that failure detection can be tested on a GPU
+ * without a fault.
+ */
+MOE_API moe_status_t moe_debug_decode_withhold(const void *hidden_states, const void *gate_up_proj,
+                                               const void *down_proj, const int32_t *top_k_index,
+                                               const float *top_k_weights, int top_k, int T, int H,
+                                               int F, int E, void *out, void *workspace,
+                                               size_t workspace_bytes, int withhold_chunk,
+                                               void *stream);
 
 /*
  * Host-input staging for a step (no operation of the method: plumbing for

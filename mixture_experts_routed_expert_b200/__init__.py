@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_W_BF16 = 0
 MOE_W_FP8_E4M3 = 1
 MOE_W_MXFP4 = 2
+WORKSPACE_HEADER_BYTES = 8192   # zero before a workspace's first use (include/moe_b200.h)
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
           4: "MOE_ERR_CUDA", 5: "MOE_ERR_TIMEOUT"}
 
@@ -31,7 +32,8 @@ EXPORTS = ("moe_abi_version", "moe_status_string", "moe_experts_workspace_size",
            "moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
            "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
            "moe_experts_shared_workspace_size", "moe_experts_with_shared",
-           "moe_experts_decode_fused", "moe_stage_inputs")
+           "moe_experts_decode_fused", "moe_stage_inputs", "moe_workspace_init",
+           "moe_workspace_status", "moe_debug_decode_withhold")
 
 
 def _load():
@@ -57,9 +59,13 @@ def _load():
     L.moe_experts_with_shared.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P,
                                           P, P, P, P, I, P, P, P, Z, P]
     L.moe_stage_inputs.argtypes = [P, P, Z, P]
+    L.moe_workspace_init.argtypes = [P, Z, P]
+    L.moe_workspace_status.argtypes = [P, I, P]
+    L.moe_debug_decode_withhold.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, I, P]
     for n in ("moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
               "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
-              "moe_experts_with_shared", "moe_experts_decode_fused", "moe_stage_inputs"):
+              "moe_experts_with_shared", "moe_experts_decode_fused", "moe_stage_inputs",
+              "moe_workspace_init", "moe_workspace_status", "moe_debug_decode_withhold"):
         getattr(L, n).restype = I
     return L
 
@@ -159,8 +165,8 @@ def _forward(name, hidden_states, gate_up_proj, down_proj, top_k_index, top_k_we
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
     decode = name in ("moe_experts_decode", "moe_experts_decode_fused")
     need = moe_experts_workspace_size(T, H, F2 // 2, E, top_k, wt, decode)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=hidden_states.device)
+    if workspace is None:   # zero-filled: the header must be zero before first use
+        workspace = torch.zeros(max(need, WORKSPACE_HEADER_BYTES), dtype=torch.uint8, device=hidden_states.device)
     rc = getattr(_lib(), name)(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
                             _ptr(top_k_index), _ptr(top_k_weights), top_k, T, H, F2 // 2, E, wt,
                             _ptr(gate_up_scale), _ptr(down_scale), _ptr(out), _ptr(workspace),
@@ -222,8 +228,8 @@ def moe_experts_with_shared(hidden_states, gate_up_proj, down_proj, top_k_index,
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden_states.device)
     need = moe_experts_shared_workspace_size(T, H, F, E, top_k, S, wt)
-    if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=hidden_states.device)
+    if workspace is None:   # zero-filled: the header must be zero before first use
+        workspace = torch.zeros(max(need, WORKSPACE_HEADER_BYTES), dtype=torch.uint8, device=hidden_states.device)
     rc = _lib().moe_experts_with_shared(
         _ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj), _ptr(top_k_index),
         _ptr(top_k_weights), top_k, T, H, F, E, wt, _ptr(gate_up_scale), _ptr(down_scale),
@@ -260,6 +266,24 @@ def moe_experts_decode_static(hidden_states, gate_up_proj, down_proj, top_k_inde
                                           _stream(stream))
     _check(rc, "moe_experts_decode_static")
     return out
+
+
+def moe_workspace_init(workspace, stream=None):
+    """Zero the workspace's 8 KiB header (needed once before first use unless
+    the workspace was allocated zero-filled)."""
+    rc = _lib().moe_workspace_init(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
+    _check(rc, "moe_workspace_init")
+    return workspace
+
+
+def moe_workspace_status(workspace, clear=False, stream=None):
+    """Status code of the calls that used `workspace` (waits for the stream):
+    MOE_OK (0) or MOE_ERR_TIMEOUT (5); clear=True also zeroes the header."""
+    rc = _lib().moe_workspace_status(_ptr(workspace), int(bool(clear)), _stream(stream))
+    if rc not in (0, 5):
+        _check(rc, "moe_workspace_status")
+    return rc
 
 
 def moe_stage_inputs(src_ptr, dst, nbytes=None, stream=None):
@@ -315,7 +339,7 @@ def moe_debug_permute(top_k_index, E, workspace=None, stream=None):
     inv = torch.empty(max(T * K, 1), dtype=torch.int32, device=dev)
     need = moe_experts_workspace_size(T, 128, 128, E, K, MOE_W_BF16, False)
     if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(max(need, WORKSPACE_HEADER_BYTES), dtype=torch.uint8, device=dev)
     rc = _lib().moe_debug_permute(_ptr(top_k_index), T, K, E, _ptr(counts), _ptr(offsets), _ptr(perm),
                                _ptr(inv), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "moe_debug_permute")

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libmoe_b200 (declared in include/moe_b200.h):
 // host-side validation, workspace layout and dispatch to the kernels.
-// Nothing here synchronises with the device or allocates device memory.
+// Nothing here allocates device memory; only moe_workspace_status waits for
+// the device (it reads the status word back).
 #include <string.h>
 
 #include <algorithm>
@@ -52,6 +53,8 @@ struct Bump {
     }
 };
 
+constexpr int32_t DEV_TIMEOUT_BIT = 1;   // the kernels' DEV_TIMEOUT status bit
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned32(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
@@ -81,10 +84,11 @@ Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t w
     };
     Workspace L;
     Bump b;
-    L.status = b.take(16);
-    // work counters of the fused MXFP4 decode kernel, next to the status word
-    // so that one clear covers both
-    L.ctr = L.status + 16;
+    L.status = 0;                       // in the header (see internal.h)
+    b.off = kWorkspaceHeaderBytes;
+    // work counters of the fused MXFP4 decode kernel (the permutation kernel
+    // clears them at the start of every call)
+    L.ctr = b.off;
     L.ctr_bytes = (wt == MOE_W_MXFP4 && fused_mxf4_fits((int)T, K))
                       ? sizeof(int32_t) * ((size_t)kFusedMaxSlots + (size_t)T * (H / 128))
                       : 0;
@@ -111,7 +115,8 @@ DecodeWorkspace decode_workspace(int T, int H, int F, int E, int K, moe_wtype_t 
     const size_t N = (size_t)T * K;
     DecodeWorkspace L;
     Bump b;
-    L.sync = b.take(sizeof(int32_t) * 4);
+    L.sync = 0;                         // in the header (see internal.h)
+    b.off = kWorkspaceHeaderBytes;
     L.h = b.take(2 * N * F);
     L.total = b.off;
     return L;
@@ -135,6 +140,12 @@ bool decode_fits(int T, int K, int H, int F) {
 constexpr int kGemvMaxSlots = 16;
 bool decode_serves(int T, int K, int H, int F, moe_wtype_t wt) {
     return wt == MOE_W_BF16 && T * K <= kGemvMaxSlots && decode_fits(T, K, H, F);
+}
+// bf16 decode calls with T <= 16, T*K <= 64 and H, F <= 2048 take the fused
+// one-kernel decode (decode_fused.cu) when the device runs its clusters.
+bool fused_decode_sizes(int T, int K, int H, int F, moe_wtype_t wt) {
+    return wt == MOE_W_BF16 && T <= kDecodeMaxT && T * K <= kDecodeMaxSlots && H <= 2048 &&
+           F <= 2048;
 }
 // Tile height of the E4M3 and MXFP4 grouped GEMMs: 16 routed rows for
 // decode-sized calls and whenever the experts average <= 6 routed rows (a
@@ -261,9 +272,12 @@ const char *moe_status_string(moe_status_t s) {
 
 size_t moe_experts_workspace_size(int T, int H, int F, int E, int K, moe_wtype_t wt, int decode) {
     if (!dims_ok(T, H, F, E, K)) return 0;
-    if (decode && decode_serves(T, K, H, F, wt))
-        return decode_workspace(T, H, F, E, K, wt).total;
-    return prefill_workspace(T, H, F, E, K, wt).total;
+    size_t need = (decode && decode_serves(T, K, H, F, wt)) ? decode_workspace(T, H, F, E, K, wt).total
+                                                           : prefill_workspace(T, H, F, E, K, wt).total;
+    // the fused decode kernel, or the path above where the device cannot run it
+    if (decode && fused_decode_sizes(T, K, H, F, wt))
+        need = std::max(need, fused_decode_workspace(T, H, F, K).total);
+    return need;
 }
 
 moe_status_t moe_experts_prefill(const void *hidden_states, const void *gate_up_proj,
@@ -292,6 +306,14 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
                                   out);
     if (s != MOE_OK || T == 0) return s;
     cudaStream_t st = (cudaStream_t)stream;
+    if (fused_decode_sizes(T, top_k, H, F, wt) && decode_fused_bf16_fits(T, H, F, top_k)) {
+        const FusedDecodeWorkspace FL = fused_decode_workspace(T, H, F, top_k);
+        if (!workspace || workspace_bytes < FL.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+            return MOE_ERR_WORKSPACE;
+        return from_cuda(launch_decode_fused_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                                  top_k_weights, T, H, F, E, top_k,
+                                                  static_cast<uint8_t *>(workspace), FL, out, st));
+    }
     if (!decode_serves(T, top_k, H, F, wt))
         return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                            top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
@@ -435,6 +457,48 @@ moe_status_t moe_debug_permute(const int32_t *top_k_index, int T, int K, int E, 
     cudaError_t e = launch_permute(top_k_index, N, E, kBNGateUp, kBNDown, ws, L, st);
     if (e == cudaSuccess) e = launch_debug_outputs(top_k_index, N, E, ws, L, counts, offsets, perm, inv, st);
     return from_cuda(e);
+}
+
+moe_status_t moe_debug_decode_withhold(const void *hidden_states, const void *gate_up_proj,
+                                       const void *down_proj, const int32_t *top_k_index,
+                                       const float *top_k_weights, int top_k, int T, int H, int F,
+                                       int E, void *out, void *workspace, size_t workspace_bytes,
+                                       int withhold_chunk, void *stream) {
+    moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                  top_k_weights, top_k, T, H, F, E, MOE_W_BF16, nullptr, nullptr,
+                                  out);
+    if (s != MOE_OK || T == 0) return s;
+    if (withhold_chunk < 0) return MOE_ERR_INVALID_ARG;
+    if (!fused_decode_sizes(T, top_k, H, F, MOE_W_BF16) || !decode_fused_bf16_fits(T, H, F, top_k))
+        return MOE_ERR_UNSUPPORTED;
+    const FusedDecodeWorkspace FL = fused_decode_workspace(T, H, F, top_k);
+    if (!workspace || workspace_bytes < FL.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return MOE_ERR_WORKSPACE;
+    return from_cuda(launch_decode_fused_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                              top_k_weights, T, H, F, E, top_k,
+                                              static_cast<uint8_t *>(workspace), FL, out,
+                                              (cudaStream_t)stream, withhold_chunk));
+}
+
+moe_status_t moe_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+    if (!workspace || workspace_bytes < kWorkspaceHeaderBytes ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(cudaMemsetAsync(workspace, 0, kWorkspaceHeaderBytes, (cudaStream_t)stream));
+}
+
+moe_status_t moe_workspace_status(void *workspace, int clear, void *stream) {
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    int32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && clear) {
+        e = cudaMemsetAsync(workspace, 0, kWorkspaceHeaderBytes, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+    return (word & DEV_TIMEOUT_BIT) ? MOE_ERR_TIMEOUT : MOE_OK;
 }
 
 moe_status_t moe_stage_inputs(const void *src, void *dst, size_t bytes, void *stream) {

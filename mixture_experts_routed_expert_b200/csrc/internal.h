@@ -21,6 +21,14 @@ constexpr int kBNFp8Decode = 16;  // the same GEMMs for a few tokens (decode ent
 constexpr int kBNMxf4Wide = 112;  // MXFP4 GEMMs with many routed rows per expert
 
 // ---- workspace layout ------------------------------------------------------
+// Every workspace starts with a header of kWorkspaceHeaderBytes: the int32
+// device status word at offset 0 and, from kWorkspaceCounterOffset, the
+// counters of the fused bf16 decode kernel.  The header is zero before a
+// workspace's first use and every call that completes leaves it so
+// (counters are reset by the kernel that used them).
+constexpr size_t kWorkspaceHeaderBytes = 8192;
+constexpr size_t kWorkspaceCounterOffset = 256;
+
 struct Workspace {
     size_t status;        // int32 device status word
     size_t ctr;           // fused MXFP4 decode: int32 work counters (cleared with the status word)
@@ -39,6 +47,21 @@ struct Workspace {
     size_t total;
 };
 Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t wt);
+
+// Fused bf16 decode (one kernel): header (status; per touched expert the
+// published h groups and the finished down rows; per (token, 32-row block)
+// the combine arrivals), then h [T*K][F] bf16 and y [T*K][H] fp32 by slot.
+struct FusedDecodeWorkspace {
+    size_t status, hdone, hused, ctr, h, y, total;
+};
+FusedDecodeWorkspace fused_decode_workspace(int T, int H, int F, int K);
+// True when the fused bf16 decode kernel serves these sizes on the current
+// device (T <= 16, T*K <= 64, H, F <= 2048 and the shared-memory plan fits).
+bool decode_fused_bf16_fits(int T, int H, int F, int K);
+cudaError_t launch_decode_fused_bf16(const void *x, const void *gate_up, const void *down,
+                                     const int32_t *idx, const float *w, int T, int H, int F,
+                                     int E, int K, uint8_t *ws, const FusedDecodeWorkspace &L,
+                                     void *out, cudaStream_t st, int withhold = -1);
 
 struct DecodeWorkspace {
     size_t sync;          // int32 status words (4)

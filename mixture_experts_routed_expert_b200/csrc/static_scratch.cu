@@ -33,7 +33,7 @@ __device__ __align__(256) uint8_t g_decode_scratch[kStaticScratchBytes];
 // The largest decode scratch (T*K <= kDecodeMaxSlots slots of h, F <= 2048
 // features, plus the status words) fits the array, so every size the decode
 // kernels accept is served.
-static_assert(256 + (size_t)kDecodeMaxSlots * 2048 * 2 <= kStaticScratchBytes,
+static_assert(kWorkspaceHeaderBytes + (size_t)kDecodeMaxSlots * 2048 * 2 <= kStaticScratchBytes,
               "static decode scratch smaller than the largest decode workspace");
 
 // Device address of g_decode_scratch in the current context.

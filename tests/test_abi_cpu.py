@@ -46,12 +46,16 @@ def test_exports_match_header(mod):
 def test_workspace_sizes(mod):
     ws = mod.moe_experts_workspace_size
     assert ws(2048, 1280, 896, 64, 6) > 2048 * 6 * (1280 * 2 + 896 * 2 + 1280 * 4)
-    assert ws(1, 1280, 896, 64, 6, decode=True) >= 6 * 896 * 2
-    # gather-GEMV decode (<= 16 slots) needs only h; larger decode calls and
+    # bf16 decode: the fused kernel's header, h (bf16) and y (fp32) by slot,
+    # and at least what the fallback kernels need
+    for T in (1, 2, 4, 8, 10):
+        d = ws(T, 1280, 896, 64, 6, decode=True)
+        assert d >= 8192 + T * 6 * (896 * 2 + 1280 * 4)
+    assert ws(11, 1280, 896, 64, 6, decode=True) == ws(11, 1280, 896, 64, 6)   # 66 slots
     # E4M3 weights run the grouped GEMMs and need the prefill workspace
-    assert ws(2, 1280, 896, 64, 6, decode=True) < ws(2, 1280, 896, 64, 6)
-    assert ws(4, 1280, 896, 64, 6, decode=True) == ws(4, 1280, 896, 64, 6)
     assert ws(1, 7168, 2048, 256, 8, 1, decode=True) == ws(1, 7168, 2048, 256, 8, 1)
+    # every workspace starts with the 8 KiB header
+    assert ws(16, 256, 256, 8, 2) > mod.WORKSPACE_HEADER_BYTES == 8192
     assert ws(16, 100, 896, 64, 6) == 0          # H % 128 != 0
     assert ws(16, 1280, 896, 0, 6) == 0          # E == 0
     assert ws(16, 1280, 896, 64, 17) == 0        # K > 16
@@ -83,6 +87,12 @@ def test_host_validation_without_gpu(mod):
     # quantiser limits
     assert L.quantize_fp8_block128(p, 4, 100, p, p, N) == 1
     assert L.quantize_fp8_block128(p, 0, 128, p, p, N) == 0
+    # workspace header helpers
+    assert L.moe_workspace_init(N, 4096, N) == 1
+    assert L.moe_workspace_init(p, 4096, N) == 1
+    assert L.moe_workspace_status(N, 0, N) == 1
+    assert L.moe_workspace_status(q, 0, N) == 1
+    assert L.moe_debug_decode_withhold(p, p, p, p, p, 6, 1, 1280, 896, 64, p, p, 1 << 30, -1, N) == 1
     # input staging: sizes in 16-byte units, aligned pointers
     assert L.moe_stage_inputs(N, N, 0, N) == 0
     assert L.moe_stage_inputs(p, p, 24, N) == 1
