@@ -164,19 +164,23 @@ MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *g
                                 size_t workspace_bytes, void *stream);
 
 /*
- * The MXFP4 decode form as one persistent kernel after the permutation
- * (row "single-kernel fusion" of the DeepGEMM Mega MoE news page: the MoE
- * steps in one kernel so that the intermediate round trips go away): gate_up
- * tiles, down tiles and the top-K combine run in the same launch, the down
- * tiles of a 16-row tile waiting (bounded) for its gate_up tiles, the last
- * down tile of a (token, 128-row block) summing that block in k order.
- * Same arguments, layouts and results as moe_experts_decode with
- * wt = MOE_W_MXFP4 and T <= 16, T * K <= 64 (otherwise MOE_ERR_UNSUPPORTED);
- * workspace from moe_experts_workspace_size(..., MOE_W_MXFP4, 1).  On B200 it
- * is not faster than moe_experts_decode's separate kernels at these sizes
- * (programmatic dependent launch already overlaps their boundaries, and each
- * down tile needs all of its rows' gate_up tiles), so moe_experts_decode
- * does not use it.
+ * The decode form as ONE kernel launch (the single-kernel fusion of the
+ * DeepGEMM Mega MoE news page: the MoE steps in one kernel so that the
+ * intermediate round trips between kernels go away).  Same arguments,
+ * layouts and results (within the parity tolerance) as moe_experts_decode;
+ * workspace from moe_experts_workspace_size(..., 1).
+ *  - bf16 weights, T <= 16, T * K <= 64, H, F <= 2048: one launch does the
+ *    expert dedup of the slots, the gate/up GEMV with SiLU*up, the down
+ *    GEMV and the fixed-order top-K combine; the CTAs that need an expert's
+ *    h wait (bounded) on a per-expert counter in the workspace header while
+ *    their down-projection rows keep streaming in.  Launched as a
+ *    programmatic dependent of the previous kernel on the stream.
+ *  - MXFP4 weights, T <= 16, T * K <= 64: one persistent kernel after the
+ *    permutation kernel (gate_up tiles, down tiles and the top-K combine;
+ *    down tiles wait, bounded, for their rows' gate_up tiles).
+ *  - anything else: MOE_ERR_UNSUPPORTED.
+ * On B200 neither form is faster than moe_experts_decode's kernels at the
+ * measured sizes, so moe_experts_decode does not use them.
  */
 MOE_API moe_status_t moe_experts_decode_fused(const void *hidden_states, const void *gate_up_proj,
                                       const void *down_proj, const int32_t *top_k_index,

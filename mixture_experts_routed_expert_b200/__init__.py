@@ -242,9 +242,10 @@ def moe_experts_with_shared(hidden_states, gate_up_proj, down_proj, top_k_index,
 
 def moe_experts_decode_fused(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                              top_k, gate_up_scale=None, down_scale=None, out=None, workspace=None,
-                             stream=None, weight_format="mxfp4"):
-    """MXFP4 decode form as one persistent kernel after the permutation
-    (gate_up, down and the combine in one launch); T <= 16, T*K <= 64."""
+                             stream=None, weight_format=None):
+    """Decode form as one kernel launch: bf16 weights (T <= 16, T*K <= 64,
+    H, F <= 2048) or MXFP4 weights (T <= 16, T*K <= 64, one persistent
+    kernel after the permutation)."""
     return _forward("moe_experts_decode_fused", hidden_states, gate_up_proj, down_proj,
                     top_k_index, top_k_weights, top_k, gate_up_scale, down_scale, out, workspace,
                     stream, weight_format)

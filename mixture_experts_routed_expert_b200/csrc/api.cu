@@ -141,8 +141,12 @@ constexpr int kGemvMaxSlots = 16;
 bool decode_serves(int T, int K, int H, int F, moe_wtype_t wt) {
     return wt == MOE_W_BF16 && T * K <= kGemvMaxSlots && decode_fits(T, K, H, F);
 }
-// bf16 decode calls with T <= 16, T*K <= 64 and H, F <= 2048 take the fused
-// one-kernel decode (decode_fused.cu) when the device runs its clusters.
+// Sizes of the one-kernel bf16 decode (decode_fused.cu), served by
+// moe_experts_decode_fused.  moe_experts_decode keeps the two-kernel GEMV
+// pair / grouped GEMMs, faster on every measured OCR-2 size (graph replay,
+// isolated / back to back, us): T=1 24.6 / 17.8 vs 26.6 / 21.6; T=2
+// 32.8 / 27.6 vs 36.9 / 30.5; T=4 (grouped) 47.1 / 42.6 vs 49.2 / 45.9;
+// T=8 (grouped) 65.5 / 57.4 vs 73.7 / 71.1.
 bool fused_decode_sizes(int T, int K, int H, int F, moe_wtype_t wt) {
     return wt == MOE_W_BF16 && T <= kDecodeMaxT && T * K <= kDecodeMaxSlots && H <= 2048 &&
            F <= 2048;
@@ -306,14 +310,6 @@ moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_p
                                   out);
     if (s != MOE_OK || T == 0) return s;
     cudaStream_t st = (cudaStream_t)stream;
-    if (fused_decode_sizes(T, top_k, H, F, wt) && decode_fused_bf16_fits(T, H, F, top_k)) {
-        const FusedDecodeWorkspace FL = fused_decode_workspace(T, H, F, top_k);
-        if (!workspace || workspace_bytes < FL.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
-            return MOE_ERR_WORKSPACE;
-        return from_cuda(launch_decode_fused_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
-                                                  top_k_weights, T, H, F, E, top_k,
-                                                  static_cast<uint8_t *>(workspace), FL, out, st));
-    }
     if (!decode_serves(T, top_k, H, F, wt))
         return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights,
                            top_k, T, H, F, E, wt, gate_up_scale, down_scale, out, workspace,
@@ -396,6 +392,17 @@ moe_status_t moe_experts_decode_fused(const void *hidden_states, const void *gat
                                   top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
                                   out);
     if (s != MOE_OK || T == 0) return s;
+    if (wt == MOE_W_BF16) {
+        if (!fused_decode_sizes(T, top_k, H, F, wt) || !decode_fused_bf16_fits(T, H, F, top_k))
+            return MOE_ERR_UNSUPPORTED;
+        const FusedDecodeWorkspace FL = fused_decode_workspace(T, H, F, top_k);
+        if (!workspace || workspace_bytes < FL.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+            return MOE_ERR_WORKSPACE;
+        return from_cuda(launch_decode_fused_bf16(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                                  top_k_weights, T, H, F, E, top_k,
+                                                  static_cast<uint8_t *>(workspace), FL, out,
+                                                  (cudaStream_t)stream));
+    }
     if (wt != MOE_W_MXFP4 || !fused_mxf4_fits(T, top_k)) return MOE_ERR_UNSUPPORTED;
     const Workspace L = prefill_workspace(T, H, F, E, top_k, wt);
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255))

@@ -1,5 +1,5 @@
-"""GPU parity of the one-kernel bf16 decode (moe_experts_decode with bf16
-weights, T <= 16, T*K <= 64) against the oracle on routings that exercise
+"""GPU parity of the one-kernel bf16 decode (moe_experts_decode_fused with
+bf16 weights, T <= 16, T*K <= 64) against the oracle on routings that exercise
 its work split: clusters with no groups (fewer feature groups than
 clusters), a touched expert split over several clusters, tokens with more
 than 8 slots on one expert, segments wider than one staging slab (64 slots
@@ -29,8 +29,9 @@ def _ref(lay):
 
 
 def _decode(moe, lay, dev, ws=None):
-    return moe.moe_experts_decode(lay.x.to(dev), lay.gate_up.to(dev), lay.down.to(dev),
-                                  lay.idx.to(dev), lay.w.to(dev), lay.idx.shape[1], workspace=ws)
+    return moe.moe_experts_decode_fused(lay.x.to(dev), lay.gate_up.to(dev), lay.down.to(dev),
+                                        lay.idx.to(dev), lay.w.to(dev), lay.idx.shape[1],
+                                        workspace=ws)
 
 
 @pytest.mark.parametrize("T,H,F,E,K", [
@@ -42,9 +43,13 @@ def _decode(moe, lay, dev, ws=None):
     (5, 2048, 2048, 16, 4),    # the largest H and F the kernel takes
 ])
 def test_fused_decode_shapes(moe, cuda_dev, T, H, F, E, K):
+    """Full outputs against the oracle; 17 tokens are refused."""
     lay = inputs.ocr2_layer(T, seed=31 * T + H, device="cpu", H=H, F=F, E=E, K=K)
     out = _decode(moe, lay, cuda_dev)
     assert_matches_oracle(out, _ref(lay), "fused decode T=%d H=%d F=%d E=%d K=%d" % (T, H, F, E, K))
+    with pytest.raises(moe.MoEError):        # 17 tokens: outside the one-kernel form
+        lay17 = inputs.ocr2_layer(17, seed=1, device="cpu", H=H, F=F, E=E, K=1)
+        _decode(moe, lay17, cuda_dev)
 
 
 def test_fused_decode_hot_expert_and_slabs(moe, cuda_dev):
@@ -72,9 +77,9 @@ def test_fused_decode_invalid_and_empty_tokens(moe, cuda_dev):
     assert torch.count_nonzero(out[3].float()) == 0
     lay.idx[:] = -1                   # nothing valid at all
     out = torch.full((6, 1280), float("nan"), dtype=torch.bfloat16, device=cuda_dev)
-    out = moe.moe_experts_decode(lay.x.to(cuda_dev), lay.gate_up.to(cuda_dev),
-                                 lay.down.to(cuda_dev), lay.idx.to(cuda_dev), lay.w.to(cuda_dev),
-                                 6, out=out)
+    out = moe.moe_experts_decode_fused(lay.x.to(cuda_dev), lay.gate_up.to(cuda_dev),
+                                       lay.down.to(cuda_dev), lay.idx.to(cuda_dev),
+                                       lay.w.to(cuda_dev), 6, out=out)
     assert torch.count_nonzero(out.float()) == 0
 
 
@@ -88,8 +93,9 @@ def test_fused_decode_workspace_reuse_is_deterministic(moe, cuda_dev):
                      dtype=torch.uint8, device=cuda_dev)
     for T, seed in ((1, 1), (4, 2), (8, 3), (1, 4), (2, 5)):
         lay = inputs.ocr2_layer(T, seed=seed, device=cuda_dev, weights_from=base)
-        a = moe.moe_experts_decode(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K, workspace=ws)
-        b = moe.moe_experts_decode(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K)
+        a = moe.moe_experts_decode_fused(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K,
+                                         workspace=ws)
+        b = moe.moe_experts_decode_fused(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K)
         assert torch.equal(a.view(torch.int16), b.view(torch.int16)), (T, seed)
     torch.cuda.synchronize()
     assert torch.count_nonzero(ws[:moe.WORKSPACE_HEADER_BYTES]) == 0

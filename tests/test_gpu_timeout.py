@@ -34,7 +34,8 @@ def test_decode_wait_expires_and_is_reported(cuda_dev, chunk):
     assert torch.count_nonzero(ws[:moe.WORKSPACE_HEADER_BYTES]) == 0
     assert moe.moe_workspace_status(ws) == 0
     # the device and the cleared workspace still serve a normal call
-    out = moe.moe_experts_decode(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K, workspace=ws)
+    out = moe.moe_experts_decode_fused(lay.x, lay.gate_up, lay.down, lay.idx, lay.w, K,
+                                       workspace=ws)
     ref = oracle.moe_forward_bf16(inputs.bf16_bits(lay.x), inputs.bf16_bits(lay.gate_up),
                                   inputs.bf16_bits(lay.down), inputs.np32(lay.idx),
                                   inputs.np32(lay.w))
