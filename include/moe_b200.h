@@ -270,6 +270,39 @@ MOE_API moe_status_t moe_experts_decode_static(const void *hidden_states, const 
                                        const void *down_scale, void *out, void *stream);
 
 /*
+ * Expert-parallel building blocks (DeepGEMM Mega MoE news page: EP dispatch
+ * and combine around the expert GEMMs; "MegaMOE adaptation for SM90" PR:
+ * dispatch to the ranks that own the experts, combine back to the tokens'
+ * rank).  With the experts sharded over ranks, a rank runs its received
+ * rows through moe_experts_rows and the tokens' rank sums the returned rows
+ * with moe_combine_rows; the exchange between them is the caller's (the
+ * Python package's expert-parallel layer uses NCCL all-to-all).
+ *
+ * moe_experts_rows: the grouped path of moe_experts_prefill without its
+ * combine.  Same arguments except `out`; on return *y_offset is the byte
+ * offset, inside `workspace`, of y [T*K][H] fp32: y[t*K+k] =
+ * w[t,k] * down_e(SiLU(gate_e x_t) * (up_e x_t)) with e = top_k_index[t,k]
+ * (rows of slots whose id is outside [0, E) are undefined).  The rows stay
+ * valid until the next call that uses the workspace.
+ */
+MOE_API moe_status_t moe_experts_rows(const void *hidden_states, const void *gate_up_proj,
+                                      const void *down_proj, const int32_t *top_k_index,
+                                      const float *top_k_weights, int top_k, int T, int H, int F,
+                                      int E, moe_wtype_t wt, const void *gate_up_scale,
+                                      const void *down_scale, void *workspace,
+                                      size_t workspace_bytes, size_t *y_offset, void *stream);
+
+/*
+ * The fixed-order top-K combine of caller rows: out[t] = bf16(sum over k
+ * ascending, ids in [0, E) only, of y[t*K+k]) (the step that ends
+ * moe_experts_prefill; "moe_local_reduction" of the MegaKernel layer table).
+ *   y [T*K][H] fp32 (16-byte aligned), top_k_index [T][K] int32,
+ *   out [T][H] bf16 (16-byte aligned), H % 128 == 0.
+ */
+MOE_API moe_status_t moe_combine_rows(const float *y, const int32_t *top_k_index, int top_k, int T,
+                                      int H, int E, void *out, void *stream);
+
+/*
  * Zeroes the 8 KiB header of a workspace (status word and counters),
  * asynchronously on `stream`; needed once before a workspace's first use
  * unless it was allocated zero-filled.  No allocation.

@@ -33,7 +33,8 @@ EXPORTS = ("moe_abi_version", "moe_status_string", "moe_experts_workspace_size",
            "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
            "moe_experts_shared_workspace_size", "moe_experts_with_shared",
            "moe_experts_decode_fused", "moe_stage_inputs", "moe_workspace_init",
-           "moe_workspace_status", "moe_debug_decode_withhold")
+           "moe_workspace_status", "moe_debug_decode_withhold", "moe_experts_rows",
+           "moe_combine_rows")
 
 
 def _load():
@@ -62,10 +63,13 @@ def _load():
     L.moe_workspace_init.argtypes = [P, Z, P]
     L.moe_workspace_status.argtypes = [P, I, P]
     L.moe_debug_decode_withhold.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, I, P]
+    L.moe_experts_rows.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, Z, P, P]
+    L.moe_combine_rows.argtypes = [P, P, I, I, I, I, P, P]
     for n in ("moe_experts_prefill", "moe_experts_decode", "moe_route_sigmoid_grouped",
               "quantize_fp8_block128", "moe_debug_permute", "moe_experts_decode_static",
               "moe_experts_with_shared", "moe_experts_decode_fused", "moe_stage_inputs",
-              "moe_workspace_init", "moe_workspace_status", "moe_debug_decode_withhold"):
+              "moe_workspace_init", "moe_workspace_status", "moe_debug_decode_withhold",
+              "moe_experts_rows", "moe_combine_rows"):
         getattr(L, n).restype = I
     return L
 
@@ -266,6 +270,46 @@ def moe_experts_decode_static(hidden_states, gate_up_proj, down_proj, top_k_inde
                                           E, wt, _ptr(gate_up_scale), _ptr(down_scale), _ptr(out),
                                           _stream(stream))
     _check(rc, "moe_experts_decode_static")
+    return out
+
+
+def moe_experts_rows(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
+                     gate_up_scale=None, down_scale=None, workspace=None, stream=None,
+                     weight_format=None):
+    """Weighted expert rows y [T*K, H] fp32, y[t*K+k] = w[t,k] * expert_e(x_t)
+    (the grouped path without its combine).  Returns a view into the
+    workspace, valid until the workspace's next use."""
+    T, H, F, E, wt = _check_forward_args(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                         top_k_weights, top_k, gate_up_scale, down_scale, None,
+                                         weight_format)
+    need = moe_experts_workspace_size(T, H, F, E, top_k, wt, False)
+    if workspace is None:
+        workspace = torch.zeros(max(need, WORKSPACE_HEADER_BYTES), dtype=torch.uint8,
+                                device=hidden_states.device)
+    off = ctypes.c_size_t(0)
+    rc = _lib().moe_experts_rows(_ptr(hidden_states), _ptr(gate_up_proj), _ptr(down_proj),
+                                 _ptr(top_k_index), _ptr(top_k_weights), top_k, T, H, F, E, wt,
+                                 _ptr(gate_up_scale), _ptr(down_scale), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), ctypes.byref(off),
+                                 _stream(stream))
+    _check(rc, "moe_experts_rows")
+    n = T * top_k * H * 4
+    return workspace[off.value:off.value + n].view(torch.float32).view(T * top_k, H)
+
+
+def moe_combine_rows(y, top_k_index, E, out=None, stream=None):
+    """out [T, H] bf16 = bf16(sum over valid k, ascending, of y[t*K+k])."""
+    T, K = top_k_index.shape
+    H = y.shape[1]
+    if tuple(y.shape) != (T * K, H) or y.dtype != torch.float32 or top_k_index.dtype != torch.int32:
+        raise ValueError("y must be [T*K, H] float32 and top_k_index [T, K] int32")
+    for t in (y, top_k_index):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=y.device)
+    rc = _lib().moe_combine_rows(_ptr(y), _ptr(top_k_index), K, T, H, E, _ptr(out), _stream(stream))
+    _check(rc, "moe_combine_rows")
     return out
 
 

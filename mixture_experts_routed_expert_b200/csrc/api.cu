@@ -192,6 +192,8 @@ moe_status_t check_common(const void *x, const void *gu, const void *dn, const i
     return MOE_OK;
 }
 
+// The grouped path; out == nullptr stops after the down GEMM, leaving the
+// weighted rows y [T*K][H] fp32 (by slot) in the workspace at L.y.
 moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const int32_t *idx,
                          const float *w, int K, int T, int H, int F, int E, moe_wtype_t wt,
                          const void *gus, const void *dns, void *out, void *ws, size_t ws_bytes,
@@ -214,7 +216,7 @@ moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const in
         else
             e = launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st, sh);
     }
-    if (e == cudaSuccess) e = launch_combine(idx, T, H, E, K, wsb, L, out, st, residual);
+    if (e == cudaSuccess && out) e = launch_combine(idx, T, H, E, K, wsb, L, out, st, residual);
     return from_cuda(e);
 }
 
@@ -485,6 +487,35 @@ moe_status_t moe_debug_decode_withhold(const void *hidden_states, const void *ga
                                               top_k_weights, T, H, F, E, top_k,
                                               static_cast<uint8_t *>(workspace), FL, out,
                                               (cudaStream_t)stream, withhold_chunk));
+}
+
+moe_status_t moe_experts_rows(const void *hidden_states, const void *gate_up_proj,
+                              const void *down_proj, const int32_t *top_k_index,
+                              const float *top_k_weights, int top_k, int T, int H, int F, int E,
+                              moe_wtype_t wt, const void *gate_up_scale, const void *down_scale,
+                              void *workspace, size_t workspace_bytes, size_t *y_offset,
+                              void *stream) {
+    if (!y_offset) return MOE_ERR_INVALID_ARG;
+    const void *dummy_out = reinterpret_cast<const void *>(uintptr_t(256));   // checked, never used
+    moe_status_t s = check_common(hidden_states, gate_up_proj, down_proj, top_k_index,
+                                  top_k_weights, top_k, T, H, F, E, wt, gate_up_scale, down_scale,
+                                  dummy_out);
+    if (s != MOE_OK) return s;
+    *y_offset = prefill_workspace(T, H, F, E, top_k, wt).y;
+    if (T == 0) return MOE_OK;
+    return run_prefill(hidden_states, gate_up_proj, down_proj, top_k_index, top_k_weights, top_k,
+                       T, H, F, E, wt, gate_up_scale, down_scale, nullptr, workspace,
+                       workspace_bytes, (cudaStream_t)stream, tile_rows_w(T, top_k, E, wt));
+}
+
+moe_status_t moe_combine_rows(const float *y, const int32_t *top_k_index, int top_k, int T, int H,
+                              int E, void *out, void *stream) {
+    if (!dims_ok(T, H, 128, E, top_k)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y || !top_k_index || !out || !aligned16(y) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(top_k_index) & 3))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_combine_rows(y, top_k_index, T, H, E, top_k, out, (cudaStream_t)stream));
 }
 
 moe_status_t moe_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {

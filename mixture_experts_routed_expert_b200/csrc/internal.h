@@ -138,6 +138,9 @@ cudaError_t launch_gemms_mxf4(const void *w13, const uint8_t *w13sf, const void 
 cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, const uint8_t *ws,
                            const Workspace &L, void *out, cudaStream_t st,
                            const void *residual = nullptr);
+// out[t] = bf16(sum over valid k, ascending, of y[t*K+k]) for caller rows y.
+cudaError_t launch_combine_rows(const float *y, const int32_t *idx, int64_t T, int H, int E, int K,
+                                void *out, cudaStream_t st);
 // idx2/w2 [T][K+S]: the K routed slots (ids outside [0,E) -> -1), then the S
 // shared ids E..E+S-1 with weight 1.
 cudaError_t launch_widen_routing(const int32_t *idx, const float *w, int64_t T, int E, int K,

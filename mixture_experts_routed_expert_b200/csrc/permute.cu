@@ -350,6 +350,13 @@ cudaError_t launch_combine(const int32_t *idx, int64_t T, int H, int E, int K, c
                     (uint2 *)out);
 }
 
+cudaError_t launch_combine_rows(const float *y, const int32_t *idx, int64_t T, int H, int E, int K,
+                                void *out, cudaStream_t st) {
+    const int64_t n = T * (H / 4);
+    return launch_k(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, true,
+                    (const float4 *)y, idx, T, H, E, K, (const uint2 *)nullptr, (uint2 *)out);
+}
+
 cudaError_t launch_widen_routing(const int32_t *idx, const float *w, int64_t T, int E, int K,
                                  int S, int32_t *idx2, float *w2, cudaStream_t st) {
     const int64_t n = T * (K + S);
