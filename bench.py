@@ -710,8 +710,11 @@ def run_only(args):
         torch.cuda.synchronize()
         print("ok", args.only, float(out.float().abs().sum()))
         return
-    T = {"decode1": 1, "decode4": 4, "prefill2048": 2048}[args.only]
+    T = {"decode1": 1, "decode4": 4, "prefill2048": 2048, "decode1_fused": 1,
+         "decode8_fused": 8}[args.only]
     fn = moe.moe_experts_prefill if args.only.startswith("prefill") else moe.moe_experts_decode
+    if args.only.endswith("_fused"):
+        fn = moe.moe_experts_decode_fused
     lay = inputs.ocr2_layer(T, seed=T, device=dev)
     flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(FLUSH_READ_BYTES // 4, dtype=torch.int32, device=dev)
@@ -838,7 +841,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048", "fp8_128", "fp8_small",
+    ap.add_argument("--only", choices=["decode1", "decode4", "prefill2048", "decode1_fused",
+                                       "decode8_fused", "fp8_128", "fp8_small",
                                        "fp8_dec_small", "fp8_big", "mxf4_small", "mxf4_dec_small",
                                        "mxf4_big"],
                     default=None,
