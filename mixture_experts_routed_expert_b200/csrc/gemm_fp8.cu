@@ -7,8 +7,9 @@
 // Grouped GEMM on tcgen05 with kind::f8f6f4 (E4M3 x E4M3 -> fp32, K = 32 per
 // instruction).  Because each 128-wide k-block has its own weight and
 // activation scale, every k-block's product goes to a TMEM "partial" buffer
-// (four in rotation; eight for 16-row tiles); epilogue warps read it and promote it into fp32
-// accumulators held in registers:
+// (four in rotation for gate_up, eight for down and for 16-row tiles);
+// epilogue warps read it and promote it into fp32 accumulators held in
+// registers (column pairs on fp32x2 arithmetic):
 //     acc[row, col] += (w_scale[row, kb] * x_scale[col, kb]) * partial[row, col]
 // while the MMA of the next k-block fills the other partial buffer.
 //   S4 (gate_up):  tile = 128 features of expert e (gate rows and up rows,
@@ -44,17 +45,13 @@ struct Cfg8 {
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
     static constexpr int PCOLS = NUM_A * BN;            // TMEM columns of one partial buffer
-    static constexpr int NPB = BN == 16 ? 8 : (GATE_UP ? 3 : 4);   // partial buffers in flight
-    // 64-row tiles keep their fp32 accumulators in TMEM after the partial
-    // buffers (registers would otherwise be exhausted and serialise the
-    // promotion); 16-row tiles keep them in registers.
-    static constexpr bool TACC = BN == 64;
-    static constexpr int ACC_COL = NPB * PCOLS;
-    static constexpr int COLS_USED = ACC_COL + (TACC ? NUM_A * BN : 0);
+    // partial buffers in flight: all of TMEM (512 columns) at 64-row tiles;
+    // the fp32 accumulators live in registers
+    static constexpr int NPB = BN == 16 ? 8 : (GATE_UP ? 4 : 8);
+    static constexpr int COLS_USED = NPB * PCOLS;
     static constexpr int TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
     static constexpr int NC = BN / 2;                   // columns per epilogue thread
-    static constexpr int CH = NC < 16 ? NC : 16;        // promotion chunk
     // 16-row tiles (one or two per CTA) stage the weight scales in shared
     // memory SG k-blocks ahead; wider tiles read them one k-block ahead.
     static constexpr bool STAGE_SCALES = BN == 16;
@@ -260,11 +257,11 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 }
                 cp_async_commit();
             };
-            float ag[NC], au[GATE_UP ? NC : 1];
+            float ag[NC], au[NC];
 #pragma unroll
             for (int j = 0; j < NC; ++j) ag[j] = 0.f;
 #pragma unroll
-            for (int j = 0; j < (GATE_UP ? NC : 1); ++j) au[j] = 0.f;
+            for (int j = 0; j < NC; ++j) au[j] = 0.f;
             float sg_next = 0.f, su_next = 0.f;
             if constexpr (C::STAGE_SCALES) {
                 issue_scales(0, 0);
@@ -303,96 +300,52 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 }
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + pb * C::PCOLS + half * NC;
-                const uint32_t tacc = tmem_base + ((uint32_t)(eg * 32) << 16) + C::ACC_COL + half * NC;
                 const float *sxk = sx + kb * BN + half * NC;   // this thread's column scales
                 // Load this thread's columns, hand the partial buffer back to
-                // the MMA warp, then promote the live 16-column chunks.
-                uint32_t pg[NC], pu[NC];
-                auto promote = [&](int c) {          // chunk c of C::CH columns
-                    if (C::CH * c < live) {          // warp-uniform
+                // the MMA warp, then promote the live column pairs:
+                // acc = (w_scale * x_scale) * partial + acc on fp32x2 (the
+                // roundings of the scalar form)
+                uint32_t pr[NC];
+                const float2 sg2 = make_float2(sg, sg), su2 = make_float2(su, su);
+                // acc[q..q+1] += (scale * x_scale[q..q+1]) * partial[q..q+1]
+                auto promote_pairs = [&](float (&acc)[NC], const float2 s2) {
 #pragma unroll
-                        for (int j = 0; j < C::CH; ++j) {
-                            const int q = C::CH * c + j;
-                            const float s = sxk[q];
-                            ag[q] = fmaf(sg * s, __uint_as_float(pg[q]), ag[q]);
-                            if (GATE_UP) au[q] = fmaf(su * s, __uint_as_float(pu[q]), au[q]);
+                    for (int c = 0; c < NC / 4; ++c) {
+                        if (4 * c < live) {          // warp-uniform
+                            const float4 s4 = *reinterpret_cast<const float4 *>(sxk + 4 * c);
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const int q = 4 * c + 2 * h2;
+                                const float2 sc = h2 == 0 ? make_float2(s4.x, s4.y) : make_float2(s4.z, s4.w);
+                                const float2 p2 = make_float2(__uint_as_float(pr[q]), __uint_as_float(pr[q + 1]));
+                                const float2 r2 = __ffma2_rn(__fmul2_rn(s2, sc), p2, make_float2(acc[q], acc[q + 1]));
+                                acc[q] = r2.x;
+                                acc[q + 1] = r2.y;
+                            }
                         }
                     }
                 };
-                if constexpr (C::TACC) {
-                    // partials of both halves, then the buffer goes back to the
-                    // MMA warp; accumulators: TMEM -> registers -> TMEM
-                    tmem_ld32(tb, pg);
-                    if (GATE_UP) tmem_ld32(tb + BN, pu);
+                auto load_partial = [&](uint32_t taddr) {
+                    if constexpr (NC == 32) tmem_ld32(taddr, pr);
+                    else tmem_ld8(taddr, pr);
                     tmem_ld_wait();
+                };
+                // gate (and down) partial, then the up partial: one 32-column
+                // load at a time keeps the live registers under the cap of ten
+                // warps; the buffer goes back to the MMA warp after the last load
+                load_partial(tb);
+                if (!GATE_UP) {
                     tc_fence_before();
                     mbar_arrive(&pempty[pb]);
-                    if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (16 * h < live) {         // warp-uniform
-                            uint32_t a_g[16], a_u[16];
-                            if (kb > 0) {
-                                tmem_ld16(tacc + 16 * h, a_g);
-                                if (GATE_UP) tmem_ld16(tacc + BN + 16 * h, a_u);
-                                tmem_ld_wait_regs16(a_g);
-                                if (GATE_UP) tmem_ld_wait_regs16(a_u);
-                            }
-                            // pairs of columns: (w_scale * x_scale) and the fma
-                            // on fp32x2, the same roundings as the scalar form
-                            const float2 sg2 = make_float2(sg, sg), su2 = make_float2(su, su);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float4 s4 = *reinterpret_cast<const float4 *>(sxk + 16 * h + 4 * i);
-#pragma unroll
-                                for (int k = 0; k < 2; ++k) {
-                                    const int j = 4 * i + 2 * k, q = 16 * h + j;
-                                    const float2 sc = k == 0 ? make_float2(s4.x, s4.y) : make_float2(s4.z, s4.w);
-                                    const float2 p2 = make_float2(__uint_as_float(pg[q]), __uint_as_float(pg[q + 1]));
-                                    const float2 a2 = kb > 0 ? make_float2(__uint_as_float(a_g[j]), __uint_as_float(a_g[j + 1]))
-                                                             : make_float2(0.f, 0.f);
-                                    const float2 r2 = __ffma2_rn(__fmul2_rn(sg2, sc), p2, a2);
-                                    a_g[j] = __float_as_uint(r2.x);
-                                    a_g[j + 1] = __float_as_uint(r2.y);
-                                    if (GATE_UP) {
-                                        const float2 pu2 = make_float2(__uint_as_float(pu[q]), __uint_as_float(pu[q + 1]));
-                                        const float2 b2 = kb > 0 ? make_float2(__uint_as_float(a_u[j]), __uint_as_float(a_u[j + 1]))
-                                                                 : make_float2(0.f, 0.f);
-                                        const float2 t2 = __ffma2_rn(__fmul2_rn(su2, sc), pu2, b2);
-                                        a_u[j] = __float_as_uint(t2.x);
-                                        a_u[j + 1] = __float_as_uint(t2.y);
-                                    }
-                                }
-                            }
-                            tmem_st16(tacc + 16 * h, a_g);
-                            if (GATE_UP) tmem_st16(tacc + BN + 16 * h, a_u);
-                        }
-                    }
-                    tmem_st_wait();
-                } else {
-                    tmem_ld8(tb, pg);
-                    if (GATE_UP) tmem_ld8(tb + BN, pu);
-                    tmem_ld_wait();
-                    tc_fence_before();
-                    mbar_arrive(&pempty[pb]);
-                    if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
-#pragma unroll
-                    for (int c = 0; c < NC / C::CH; ++c) promote(c);
                 }
-            }
-            if constexpr (C::TACC) {
-                const uint32_t tacc = tmem_base + ((uint32_t)(eg * 32) << 16) + C::ACC_COL + half * NC;
-                uint32_t r[NC];
-                tmem_ld32(tacc, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < NC; ++j) ag[j] = __uint_as_float(r[j]);
+                promote_pairs(ag, sg2);
                 if (GATE_UP) {
-                    tmem_ld32(tacc + BN, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < NC; ++j) au[j] = __uint_as_float(r[j]);
+                    load_partial(tb + BN);
+                    tc_fence_before();
+                    mbar_arrive(&pempty[pb]);
+                    promote_pairs(au, su2);
                 }
+                if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
             }
             if (GATE_UP) {
                 // h = bf16(SiLU(g) * u) for this row (feature) and NC routed rows
