@@ -19,10 +19,13 @@
 //     of two with max|h|/scale <= 448, codes E4M3 -> hq [N][F], hs [N][F/128].
 //   S5 (down):  tile = 128 hidden rows x up to BN routed rows;
 //     y[slot, j] = w[slot] * acc  (fp32, by original slot; combined later).
-// Warp roles as in the bf16 kernel: warp 0 TMA producer, warp 1 TMEM
-// allocation + MMA issue, warps 2-9 promotion and epilogue (two warps per TMEM
-// lane quarter, each owning BN/2 of the BN columns; promotion skips 16-column
-// chunks past the tile's routed rows).
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocation + MMA issue, for
+// gate_up with warp 10 (warp 1 the gate MMAs, warp 10 the up MMAs of every
+// stage: one thread issuing all eight MMAs of a k-block paced the pipeline,
+// ~85 SM cycles per small tcgen05.mma against ~32 of tensor work), warps 2-9
+// promotion and epilogue (two warps per TMEM lane quarter, each owning BN/2
+// of the BN columns; promotion skips 16-column chunks past the tile's routed
+// rows).
 #include "common.cuh"
 #include "gemm_common.cuh"
 #include "internal.h"
@@ -32,13 +35,14 @@ namespace moe {
 namespace {
 
 constexpr int kEpi8 = 8;
-constexpr int kThreads8 = 64 + 32 * kEpi8;
+constexpr int kMmaWarp2 = 2 + kEpi8;            // gate_up: the warp issuing the up MMAs
 constexpr int kMaxKB8 = 128;          // k-blocks (of 128) per row supported
 
 template <bool GATE_UP, int BN>
 struct Cfg8 {
     static_assert(BN == 64 || BN == 16, "one epilogue thread owns 32 or 8 columns");
     static constexpr int NUM_A = GATE_UP ? 2 : 1;
+    static constexpr int THREADS = 64 + 32 * kEpi8 + (GATE_UP ? 32 : 0);
     static constexpr int MAX_STAGES = 12;               // ring depth: chosen at launch to fill smem
     static constexpr int BOX = BN < 32 ? BN : 32;       // routed rows per TMA box
     static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 e4m3
@@ -87,7 +91,7 @@ __device__ __forceinline__ void epi_sync() {
 }
 
 template <bool GATE_UP, int BN>
-__global__ void __launch_bounds__(kThreads8, 1)
+__global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
     grouped_gemm_fp8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, const Gemm8Args args) {
     using C = Cfg8<GATE_UP, BN>;
@@ -105,7 +109,7 @@ __global__ void __launch_bounds__(kThreads8, 1)
     float *wsc = reinterpret_cast<float *>(smem + (size_t)NST * C::STAGE_BYTES + 1024);  // [2][NUM_A][128][SG+1]
     float *sx = wsc + C::WSC_FLOATS;                                      // [KB][BN]
     float *amax_s = sx + BN * args.KB;                                    // [4][BN]
-    float *scale_s = amax_s + 4 * BN;                                     // [BN]
+    float *scale_s = amax_s + 4 * BN;                                     // [BN] 1 / h scale
     int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + BN);
     int32_t *s_tiles = s_off + (args.E + 1);
     const int KB = args.KB;
@@ -114,10 +118,10 @@ __global__ void __launch_bounds__(kThreads8, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], C::NUM_A);   // a commit per MMA-issuing warp
         }
         for (int b = 0; b < C::NPB; ++b) {
-            mbar_init(&pfull[b], 1);
+            mbar_init(&pfull[b], C::NUM_A);
             mbar_init(&pempty[b], 32 * kEpi8);
         }
         *abort_flag = 0;
@@ -188,8 +192,11 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
                     atomicOr(args.status, DEV_TIMEOUT);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || (GATE_UP && warp == kMmaWarp2)) {
         if (lane == 0) {
+            // operand r: the gate (r = 0) or up (r = 1) weight tile and its
+            // half of the partial buffer
+            const int r = warp == 1 ? 0 : 1;
             int stage = 0, pb = 0;
             uint32_t phase = 0, pphase = 0;
             bool ok = true;
@@ -201,15 +208,11 @@ __global__ void __launch_bounds__(kThreads8, 1)
                         !mbar_wait(&pempty[pb], pphase ^ 1, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(ring + stage * C::STAGE_BYTES);
-                    const uint64_t da = sdesc_sw128(sa);
-                    const uint64_t da2 = sdesc_sw128(sa + C::A_BYTES);
+                    const uint64_t da = sdesc_sw128(sa + r * C::A_BYTES);
                     const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES);
-                    const uint32_t d = tmem_base + pb * C::PCOLS;
+                    const uint32_t d = tmem_base + pb * C::PCOLS + r * BN;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        mma_e4m3_ss(d, da + 2 * k, db + 2 * k, idesc, k > 0);
-                        if (GATE_UP) mma_e4m3_ss(d + BN, da2 + 2 * k, db + 2 * k, idesc, k > 0);
-                    }
+                    for (int k = 0; k < 4; ++k) mma_e4m3_ss(d, da + 2 * k, db + 2 * k, idesc, k > 0);
                     mma_commit(&empty[stage]);
                     mma_commit(&pfull[pb]);
                     if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -230,16 +233,40 @@ __global__ void __launch_bounds__(kThreads8, 1)
         int pb = 0;
         uint32_t pphase = 0;
         bool ok = true;
+        // activation scales of a tile's routed rows -> sx[kb][column], by
+        // asynchronous 4-byte copies (64-row tiles: the next tile's are
+        // requested as soon as every warp is done with the current ones, so
+        // that they arrive during the tile's quantisation / y stores)
+        auto stage_sx = [&](const Tile &tn) {   // warp ew: k-blocks ew, ew+8, ...; lanes: rows
+            for (int kb = ew; kb < KB; kb += kEpi8)
+                for (int c = lane; c < tn.nrows; c += 32)
+                    cp_async4(sx + kb * BN + c, args.xscale + (size_t)(tn.row0 + c) * KB + kb);
+            cp_async_commit();
+        };
+        if constexpr (!C::STAGE_SCALES) {
+            if ((int)blockIdx.x < total) stage_sx(decode_tile(blockIdx.x, s_off, s_tiles, args.E, args.MT, BN));
+        }
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
-            // activation scales of this tile's routed rows
-            epi_sync();
-            for (int i = et; i < t.nrows * KB; i += 32 * kEpi8) {
-                const int c = i / KB, kb = i - c * KB;
-                sx[kb * BN + c] = __ldg(args.xscale + (size_t)(t.row0 + c) * KB + kb);
+            if constexpr (C::STAGE_SCALES) {
+                epi_sync();
+                for (int kb = ew; kb < KB; kb += kEpi8)
+                    for (int c = lane; c < t.nrows; c += 32)
+                        sx[kb * BN + c] = __ldg(args.xscale + (size_t)(t.row0 + c) * KB + kb);
+                epi_sync();
             }
-            epi_sync();
             const int live = t.nrows - half * NC;   // columns of this thread that hold routed rows
+            // down: the slot and router weight of column half*NC + lane (NC <= 32),
+            // for the y stores at the end of the tile
+            int my_slot = 0;
+            float my_w = 0.f;
+            if (!GATE_UP) {
+                const int c = half * NC + lane;
+                if (lane < NC && c < t.nrows) {
+                    my_slot = __ldg(args.perm + t.row0 + c);
+                    my_w = __ldg(args.topw + my_slot);
+                }
+            }
             // Weight scales of the tile's 128 rows: with STAGE_SCALES they
             // arrive in shared memory SG k-blocks at a time, one group ahead
             // (asynchronous copies); otherwise each is read one k-block ahead.
@@ -268,6 +295,8 @@ __global__ void __launch_bounds__(kThreads8, 1)
             } else {
                 sg_next = __ldg(wsg);
                 if (GATE_UP) su_next = __ldg(wsu);
+                cp_async_wait<0>();                  // this thread's sx copies have landed
+                epi_sync();                          // and every thread's
             }
             for (int kb = 0; kb < KB; ++kb) {
                 const int grp = kb / C::SG, q = kb - grp * C::SG, buf = grp & 1;
@@ -347,61 +376,52 @@ __global__ void __launch_bounds__(kThreads8, 1)
                 }
                 if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
             }
+            if constexpr (!C::STAGE_SCALES) {
+                epi_sync();                          // every warp is done with sx
+                if (w + (int)gridDim.x < total)
+                    stage_sx(decode_tile(w + gridDim.x, s_off, s_tiles, args.E, args.MT, BN));
+            }
             if (GATE_UP) {
-                // h = bf16(SiLU(g) * u) for this row (feature) and NC routed rows
+                // h = bf16(SiLU(g) * u) for this row (feature) and NC routed
+                // rows (SiLU with the fast division, as the bf16 epilogue)
 #pragma unroll
-                for (int j = 0; j < NC; ++j)
-                    ag[j] = __bfloat162float(__float2bfloat16_rn(silu_f(ag[j]) * au[j]));
-                // column max of |h| over this warp's 32 rows, 32 columns at a
-                // time: lane l ends with column l of the group
-#pragma unroll
-                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
-                    float v[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = 32 * grp + j < NC ? fabsf(ag[32 * grp + j]) : 0.f;
-#pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) {
-#pragma unroll
-                        for (int i = 0; i < o; ++i) {
-                            const bool upper = (lane & o) != 0;
-                            const float send = upper ? v[i] : v[i + o];
-                            const float keep = upper ? v[i + o] : v[i];
-                            v[i] = fmaxf(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
-                        }
-                    }
-                    if (32 * grp + lane < NC) amax_s[eg * BN + half * NC + 32 * grp + lane] = v[0];
+                for (int j = 0; j < NC; ++j) {
+                    const float g = ag[j];
+                    ag[j] = __bfloat162float(__float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * au[j]));
                 }
+                // column max of |h| over this warp's 32 rows: |h| >= 0, so the
+                // fp32 bit patterns order like the values and one redux.sync
+                // per column gives its max; lane j keeps column j
+                float cmax = 0.f;
+#pragma unroll
+                for (int j = 0; j < NC; ++j) {
+                    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(fabsf(ag[j])));
+                    if (lane == j) cmax = __uint_as_float(m);
+                }
+                if (lane < NC) amax_s[eg * BN + half * NC + lane] = cmax;
                 epi_sync();
                 if (et < BN) {
                     const float m = fmaxf(fmaxf(amax_s[et], amax_s[BN + et]),
                                           fmaxf(amax_s[2 * BN + et], amax_s[3 * BN + et]));
                     const int k = fp8_block_exp(m);
-                    scale_s[et] = pow2f(k);
+                    scale_s[et] = 1.0f / pow2f(k);   // codes are h * (1 / scale), once per column
                     if (et < t.nrows) args.hs[(size_t)(t.row0 + et) * (args.F / 128) + t.m] = pow2f(k);
                 }
                 epi_sync();
                 uint8_t *hp = args.hq + (size_t)(t.row0 + half * NC) * args.F + t.m * kBM + row;
 #pragma unroll
-                for (int j = 0; j < NC; ++j) {
-                    if (j < live) {
-                        const float inv = 1.0f / scale_s[half * NC + j];
-                        hp[(size_t)j * args.F] = (uint8_t)(e4m3x2(ag[j] * inv, 0.f) & 0xFF);
-                    }
-                }
+                for (int j = 0; j < NC; ++j)
+                    if (j < live)
+                        hp[(size_t)j * args.F] = (uint8_t)(e4m3x2(ag[j] * scale_s[half * NC + j], 0.f) & 0xFF);
             } else {
+                // y[slot, row] = w[slot] * acc; lane l's slot and weight were
+                // read at the start of the tile
                 float *yp = args.y + t.m * kBM + row;
 #pragma unroll
-                for (int grp = 0; grp < (NC + 31) / 32; ++grp) {
-                    const int c = half * NC + 32 * grp + lane;
-                    const int my_slot = (c < t.nrows) ? __ldg(args.perm + t.row0 + c) : 0;
-                    const float my_w = (c < t.nrows) ? __ldg(args.topw + my_slot) : 0.f;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
-                        const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
-                        if (32 * grp + j < NC && 32 * grp + j < live)
-                            yp[(size_t)slot * args.H] = wj * ag[32 * grp + j];
-                    }
+                for (int j = 0; j < NC; ++j) {
+                    const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                    const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                    if (j < live) yp[(size_t)slot * args.H] = wj * ag[j];
                 }
             }
         }
@@ -427,7 +447,7 @@ cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &a2, const CUten
     if (need > kSmemMax) return cudaErrorInvalidValue;
     const cudaError_t e = enable_max_dyn_smem((const void *)grouped_gemm_fp8<GATE_UP, BN>, attr_done);
     if (e != cudaSuccess) return e;
-    return launch_k(grouped_gemm_fp8<GATE_UP, BN>, dim3(num_sms()), dim3(kThreads8), need, st, true,
+    return launch_k(grouped_gemm_fp8<GATE_UP, BN>, dim3(num_sms()), dim3(C::THREADS), need, st, true,
                     a, a2, b, a8);
 }
 
