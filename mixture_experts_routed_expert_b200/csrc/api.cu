@@ -204,7 +204,11 @@ moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const in
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     const int64_t N = (int64_t)T * K;
     const bool fp8 = (wt != MOE_W_BF16);   // E4M3 activations (E4M3 or MXFP4 weights)
-    cudaError_t e = fp8 ? launch_permute_gather(x, idx, N, K, H, E, bn8, bn8, wt, wsb, L, st)
+    // E4M3 weights: 128-row down tiles with 64-row gate_up tiles once the
+    // experts average 32 routed rows or more (below that the narrower tiles
+    // keep more stages of weights in flight)
+    const int bn8_d = (wt == MOE_W_FP8_E4M3 && bn8 == kBNFp8 && N >= (int64_t)32 * E) ? kBNFp8DownWide : bn8;
+    cudaError_t e = fp8 ? launch_permute_gather(x, idx, N, K, H, E, bn8, bn8_d, wt, wsb, L, st)
                         : launch_permute_gather(x, idx, N, K, H, E, kBNGateUp, kBNDown, wt, wsb, L, st);
     if (e == cudaSuccess) {
         if (wt == MOE_W_MXFP4)
@@ -212,7 +216,8 @@ moe_status_t run_prefill(const void *x, const void *gu, const void *dn, const in
                                   static_cast<const uint8_t *>(dns), w, T, H, F, E, K, bn8, wsb, L, st);
         else if (fp8)
             e = launch_gemms_fp8(gu, static_cast<const float *>(gus), dn,
-                                 static_cast<const float *>(dns), w, T, H, F, E, K, bn8, wsb, L, st, sh);
+                                 static_cast<const float *>(dns), w, T, H, F, E, K, bn8, bn8_d, wsb, L, st,
+                                 sh);
         else
             e = launch_gemms_bf16(gu, dn, w, T, H, F, E, K, wsb, L, st, sh);
     }

@@ -40,18 +40,19 @@ constexpr int kMaxKB8 = 128;          // k-blocks (of 128) per row supported
 
 template <bool GATE_UP, int BN>
 struct Cfg8 {
-    static_assert(BN == 64 || BN == 16, "one epilogue thread owns 32 or 8 columns");
+    static_assert(BN == 64 || BN == 16 || (!GATE_UP && BN == 128),
+                  "one epilogue thread owns 32 or 8 columns (64 of the down GEMM's wide tiles)");
     static constexpr int NUM_A = GATE_UP ? 2 : 1;
     static constexpr int THREADS = 64 + 32 * kEpi8 + (GATE_UP ? 32 : 0);
     static constexpr int MAX_STAGES = 12;               // ring depth: chosen at launch to fill smem
-    static constexpr int BOX = BN < 32 ? BN : 32;       // routed rows per TMA box
+    static constexpr int BOX = BN < 32 ? BN : (BN == 128 ? 64 : 32);   // routed rows per TMA box
     static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 e4m3
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
     static constexpr int PCOLS = NUM_A * BN;            // TMEM columns of one partial buffer
     // partial buffers in flight: all of TMEM (512 columns) at 64-row tiles;
     // the fp32 accumulators live in registers
-    static constexpr int NPB = BN == 16 ? 8 : (GATE_UP ? 4 : 8);
+    static constexpr int NPB = 512 / PCOLS < 8 ? 512 / PCOLS : 8;
     static constexpr int COLS_USED = NPB * PCOLS;
     static constexpr int TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
@@ -256,16 +257,22 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                 epi_sync();
             }
             const int live = t.nrows - half * NC;   // columns of this thread that hold routed rows
-            // down: the slot and router weight of column half*NC + lane (NC <= 32),
+            // down: the slots and router weights of columns half*NC + 32*g + lane,
             // for the y stores at the end of the tile
-            int my_slot = 0;
-            float my_w = 0.f;
-            if (!GATE_UP) {
-                const int c = half * NC + lane;
-                if (lane < NC && c < t.nrows) {
-                    my_slot = __ldg(args.perm + t.row0 + c);
-                    my_w = __ldg(args.topw + my_slot);
-                }
+            constexpr int NG = (NC + 31) / 32;
+            int my_slot[NG];
+            float my_w[NG];
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                my_slot[g] = 0;
+                my_w[g] = 0.f;
+                const int c = half * NC + 32 * g + lane;
+                if (!GATE_UP && 32 * g + lane < NC && c < t.nrows) my_slot[g] = __ldg(args.perm + t.row0 + c);
+            }
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                const int c = half * NC + 32 * g + lane;
+                if (!GATE_UP && 32 * g + lane < NC && c < t.nrows) my_w[g] = __ldg(args.topw + my_slot[g]);
             }
             // Weight scales of the tile's 128 rows: with STAGE_SCALES they
             // arrive in shared memory SG k-blocks at a time, one group ahead
@@ -355,8 +362,14 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                     }
                 };
                 auto load_partial = [&](uint32_t taddr) {
-                    if constexpr (NC == 32) tmem_ld32(taddr, pr);
-                    else tmem_ld8(taddr, pr);
+                    if constexpr (NC == 64) {        // both halves behind one wait
+                        tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(pr));
+                        tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(pr + 32));
+                    } else if constexpr (NC == 32) {
+                        tmem_ld32(taddr, pr);
+                    } else {
+                        tmem_ld8(taddr, pr);
+                    }
                     tmem_ld_wait();
                 };
                 // gate (and down) partial, then the up partial: one 32-column
@@ -419,8 +432,8 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                 float *yp = args.y + t.m * kBM + row;
 #pragma unroll
                 for (int j = 0; j < NC; ++j) {
-                    const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
-                    const float wj = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                    const int slot = __shfl_sync(0xFFFFFFFFu, my_slot[j / 32], j % 32);
+                    const float wj = __shfl_sync(0xFFFFFFFFu, my_w[j / 32], j % 32);
                     if (j < live) yp[(size_t)slot * args.H] = wj * ag[j];
                 }
             }
@@ -456,10 +469,14 @@ cudaError_t launch_one8(const CUtensorMap &a, const CUtensorMap &a2, const CUten
 
 cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
                              const float *topw, int64_t T, int H, int F, int E, int K, int bn,
-                             uint8_t *ws, const Workspace &L, cudaStream_t st, const SharedSet &sh) {
+                             int bn_d, uint8_t *ws, const Workspace &L, cudaStream_t st,
+                             const SharedSet &sh) {
     if (H / 128 > kMaxKB8 || F / 128 > kMaxKB8) return cudaErrorInvalidValue;
     if (bn != kBNFp8 && bn != kBNFp8Decode) return cudaErrorInvalidValue;
+    if (bn_d != bn && !(bn == kBNFp8 && bn_d == kBNFp8DownWide)) return cudaErrorInvalidValue;
     const int box = bn < 32 ? bn : 32;
+    // down: 128-row tiles (64-row boxes), or the gate_up tile rows
+    const int box_d = bn_d == kBNFp8DownWide ? Cfg8<false, kBNFp8DownWide>::BOX : box;
     const uint64_t N = (uint64_t)T * K;
     CUtensorMap ta, tb, tc, td, ta2, tc2;
     const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -467,7 +484,7 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     if (!make_tmap(&ta, U8, 1, w13, (uint64_t)E_split * 2 * F, H, kBM) ||
         !make_tmap(&tb, U8, 1, ws + L.xperm, N, H, box) ||
         !make_tmap(&tc, U8, 1, w2, (uint64_t)E_split * H, F, kBM) ||
-        !make_tmap(&td, U8, 1, ws + L.h, N, F, box))
+        !make_tmap(&td, U8, 1, ws + L.h, N, F, box_d))
         return cudaErrorInvalidValue;
     if (sh.S > 0) {
         if (!make_tmap(&ta2, U8, 1, sh.gate_up, (uint64_t)sh.S * 2 * F, H, kBM) ||
@@ -516,7 +533,8 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     }
     const cudaError_t err = launch_one8<true, kBNFp8>(ta, ta2, tb, a1, st);
     if (err != cudaSuccess) return err;
-    return launch_one8<false, kBNFp8>(tc, tc2, td, a2, st);
+    return bn_d == kBNFp8DownWide ? launch_one8<false, kBNFp8DownWide>(tc, tc2, td, a2, st)
+                                  : launch_one8<false, kBNFp8>(tc, tc2, td, a2, st);
 }
 
 }  // namespace moe

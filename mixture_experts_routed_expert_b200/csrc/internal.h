@@ -18,6 +18,7 @@ constexpr int kBNGateUp = 128;    // routed rows (tokens) per gate_up tile
 constexpr int kBNDown = 256;      // routed rows per down tile
 constexpr int kBNFp8 = 64;        // routed rows per tile of both E4M3 GEMMs
 constexpr int kBNFp8Decode = 16;  // the same GEMMs for a few tokens (decode entry)
+constexpr int kBNFp8DownWide = 128;  // E4M3 down GEMM tiles with 64-row gate_up tiles
 constexpr int kBNMxf4Wide = 112;  // MXFP4 GEMMs with many routed rows per expert
 
 // ---- workspace layout ------------------------------------------------------
@@ -116,10 +117,11 @@ cudaError_t launch_gemms_bf16(const void *gate_up, const void *down, const float
                               int H, int F, int E, int K, uint8_t *ws, const Workspace &L,
                               cudaStream_t st, const SharedSet &sh = SharedSet());
 // E counts the routed and the shared experts (sh.S of them, the last ids).
-// bn: kBNFp8 or kBNFp8Decode; must match the tile prefixes of the permutation.
+// bn: gate_up tile rows, kBNFp8 or kBNFp8Decode; bn_d: down tile rows, bn or
+// (with kBNFp8) kBNFp8DownWide; both must match the permutation's tile prefixes.
 cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2, const float *w2s,
                              const float *topw, int64_t T, int H, int F, int E, int K, int bn,
-                             uint8_t *ws, const Workspace &L, cudaStream_t st,
+                             int bn_d, uint8_t *ws, const Workspace &L, cudaStream_t st,
                              const SharedSet &sh = SharedSet());
 // residual: optional [T][H] bf16 added after the slot sum (nullptr: none).
 // The fused MXFP4 decode kernel (one launch for T <= kFusedMaxT,
