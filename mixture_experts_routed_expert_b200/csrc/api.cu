@@ -103,6 +103,8 @@ Workspace prefill_workspace(int64_t T, int H, int F, int E, int K, moe_wtype_t w
     L.xscale = b.take(scale_bytes(H));
     L.h = b.take(eb * (size_t)N * F);
     L.hscale = b.take(scale_bytes(F));
+    L.xsb = b.take(wt == MOE_W_FP8_E4M3 ? (size_t)N * align_up(H / 128, 16) : 0);
+    L.hsb = b.take(wt == MOE_W_FP8_E4M3 ? (size_t)N * align_up(F / 128, 16) : 0);
     L.y = b.take(sizeof(float) * (size_t)N * H);
     L.total = b.off;
     return L;

@@ -191,6 +191,10 @@ __host__ __device__ constexpr uint32_t idesc_mxf4_e4m3(int M, int N) {
     return (5u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
            ((uint32_t)(M >> 4) << 24);
 }
+// The same instruction with E4M3 A and B (format 0 both).
+__host__ __device__ constexpr uint32_t idesc_e4m3_bs(int M, int N) {
+    return ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_sf_ids(uint32_t a_id, uint32_t b_id) {
     return (a_id << 29) | (b_id << 4);
 }

@@ -48,12 +48,22 @@ struct Cfg8 {
     static constexpr int BOX = BN < 32 ? BN : (BN == 128 ? 64 : 32);   // routed rows per TMA box
     static constexpr int A_BYTES = kBM * 128;           // 128 rows x 128 e4m3
     static constexpr int B_BYTES = BN * 128;
-    static constexpr int STAGE_BYTES = NUM_A * A_BYTES + B_BYTES;
+    // BS: the power-of-two activation scales ride on the MMA as E8M0 block
+    // scales (kind::mxf8f6f4.block_scale, E4M3 x E4M3, the weights at scale
+    // 1): the tensor cores return x_scale * partial exactly, and the
+    // promotion multiplies by the weight scale alone.  The 16-row tiles keep
+    // kind::f8f6f4 and the promotion by both scales.
+    static constexpr bool BS = BN != 16;
+    static constexpr int SFB_OFF = NUM_A * A_BYTES + B_BYTES;   // a stage's activation-scale block (BS)
+    static constexpr int STAGE_BYTES = BS ? (SFB_OFF + 512 + 1023) / 1024 * 1024 : NUM_A * A_BYTES + B_BYTES;
     static constexpr int PCOLS = NUM_A * BN;            // TMEM columns of one partial buffer
-    // partial buffers in flight: all of TMEM (512 columns) at 64-row tiles;
+    // per MMA warp (BS): 4 TMEM columns of weight scales, 4 of activation scales
+    static constexpr int SF_COLS = BS ? 8 * NUM_A : 0;
+    // partial buffers in flight: the rest of TMEM's 512 columns (up to 8);
     // the fp32 accumulators live in registers
-    static constexpr int NPB = 512 / PCOLS < 8 ? 512 / PCOLS : 8;
-    static constexpr int COLS_USED = NPB * PCOLS;
+    static constexpr int NPB = (512 - SF_COLS) / PCOLS < 8 ? (512 - SF_COLS) / PCOLS : 8;
+    static constexpr int SF_COL = NPB * PCOLS;
+    static constexpr int COLS_USED = NPB * PCOLS + SF_COLS;
     static constexpr int TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
     static constexpr int NC = BN / 2;                   // columns per epilogue thread
@@ -62,9 +72,14 @@ struct Cfg8 {
     static constexpr bool STAGE_SCALES = BN == 16;
     static constexpr int SG = 8;                        // k-blocks per weight-scale group
     static constexpr int WSC_FLOATS = STAGE_SCALES ? 2 * NUM_A * kBM * (SG + 1) : 0;
+    // after the ring: barriers (1 KB); BS: the unit weight-scale block (1 KB)
+    // and the producer's table of the tile's activation scales [BN][KB];
+    // otherwise the staged weight scales and the epilogue's [KB][BN] table;
+    // then the h amax / scale arrays and the tile prefixes
     static size_t smem_bytes(int E, int KB, int stages) {
-        return 1024 + (size_t)stages * STAGE_BYTES + 1024 + sizeof(float) * WSC_FLOATS + sizeof(float) * BN * KB +
-               sizeof(float) * 5 * BN + 2 * sizeof(int) * (E + 1) + 64;
+        const size_t table = BS ? 2 * (size_t)BN * ((KB + 15) & ~15) : sizeof(float) * BN * KB;
+        return 1024 + (size_t)stages * STAGE_BYTES + 1024 + (BS ? 1024 : 0) + sizeof(float) * WSC_FLOATS +
+               table + sizeof(float) * 5 * BN + 2 * sizeof(int) * (E + 1) + 64;
     }
 };
 
@@ -76,8 +91,11 @@ struct Gemm8Args {
     const float *wscale;     // [E_split * rows][KB] weight scales
     const float *wscale2;    // [(E - E_split) * rows][KB] weight scales of the second set
     const float *xscale;     // [N][KB] activation scales of the routed rows
+    const uint8_t *xsb;      // BS: the same as E8M0 bytes, rows of KBp bytes
+    int KBp;                 // round16(KB)
     uint8_t *hq;             // gate_up: [N][F] e4m3
     float *hs;               // gate_up: [N][F/128]
+    uint8_t *hsb;            // gate_up (BS): the h scales' E8M0 bytes, rows of round16(F/128)
     int F;
     float *y;                // down: [T*K][H]
     int H;
@@ -105,11 +123,15 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
     uint64_t *empty = full + C::MAX_STAGES;
     uint64_t *pfull = empty + C::MAX_STAGES;
     uint64_t *pempty = pfull + C::NPB;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pempty + C::NPB);
+    uint64_t *tbar = pempty + C::NPB;                                     // BS: the two tables' barriers
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tbar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *wsc = reinterpret_cast<float *>(smem + (size_t)NST * C::STAGE_BYTES + 1024);  // [2][NUM_A][128][SG+1]
-    float *sx = wsc + C::WSC_FLOATS;                                      // [KB][BN]
-    float *amax_s = sx + BN * args.KB;                                    // [4][BN]
+    uint32_t *asf = reinterpret_cast<uint32_t *>(smem + (size_t)NST * C::STAGE_BYTES + 1024);   // BS: 512 B
+    float *wsc = reinterpret_cast<float *>(smem + (size_t)NST * C::STAGE_BYTES + 1024 + (C::BS ? 1024 : 0));  // [2][NUM_A][128][SG+1]
+    float *sx = wsc + C::WSC_FLOATS;              // [KB][BN] (epilogue; not BS)
+    uint8_t *tbl = reinterpret_cast<uint8_t *>(sx);   // BS: two [BN][KBp] byte tables (producer)
+    float *amax_s = C::BS ? reinterpret_cast<float *>(tbl + 2 * (size_t)BN * args.KBp)
+                          : sx + BN * args.KB;                            // [4][BN]
     float *scale_s = amax_s + 4 * BN;                                     // [BN] 1 / h scale
     int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + BN);
     int32_t *s_tiles = s_off + (args.E + 1);
@@ -125,8 +147,15 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
             mbar_init(&pfull[b], C::NUM_A);
             mbar_init(&pempty[b], 32 * kEpi8);
         }
+        mbar_init(&tbar[0], 1);
+        mbar_init(&tbar[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
+    }
+    if (C::BS && threadIdx.x < 128) {
+        // the weights' block scales: 2^0 for every row and 32-element slice
+        asf[threadIdx.x] = 0x7F7F7F7Fu;
+        fence_proxy_async_smem();
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmA);
@@ -150,28 +179,74 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
     pdl_launch_dependents();
 
     if (warp == 0) {
-        if (lane == 0) {
-            // weight tiles: evict-first when only this tile reads them, kept
-            // (evict-last) when the expert's other routed-row tiles, running
-            // on neighbouring SMs at the same time, read them too
-            const uint64_t pol_once = policy_evict_first();
-            const uint64_t pol_x = policy_evict_last();
-            int stage = 0, armed[C::MAX_STAGES];
-            uint32_t phase = 0;
-            for (int s = 0; s < C::MAX_STAGES; ++s) armed[s] = -1;
-            bool ok = true;
-            for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-                const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
-                const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
-                const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
-                const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * C::BOX * 128;
-                const bool second = t.e >= args.E_split;
-                const CUtensorMap *mA = second ? &tmA2 : &tmA;
-                const int arow = (second ? t.e - args.E_split : t.e) * args.a_rows_per_expert + t.m * kBM;
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
-                    uint8_t *sA = ring + stage * C::STAGE_BYTES;
-                    uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
+        // weight tiles: evict-first when only this tile reads them, kept
+        // (evict-last) when the expert's other routed-row tiles, running on
+        // neighbouring SMs at the same time, read them too.  Lane 0 waits and
+        // issues the copies; with BS the whole warp stages the tile's
+        // activation scales (asynchronous copies into sx[row][kb]) and writes
+        // each stage's block of E8M0 scale bytes -- the exponent field of the
+        // power-of-two scale -- in the layout tcgen05.cp 32x128b.warpx4 reads
+        // (row n at word (n % 32) * 4 + n / 32, the byte repeated for the
+        // four 32-element slices; rows past the tile at 2^0).
+        const uint64_t pol_once = policy_evict_first();
+        const uint64_t pol_x = policy_evict_last();
+        int stage = 0, armed[C::MAX_STAGES];
+        uint32_t phase = 0;
+        for (int s = 0; s < C::MAX_STAGES; ++s) armed[s] = -1;
+        bool ok = true;
+        // BS: the tile's E8M0 scale bytes arrive with one bulk copy into one of
+        // two tables, the next tile's requested as the current one is ready
+        const int KBp = args.KBp;
+        uint32_t tarmed = 0;                  // table loads issued and not yet waited for
+        uint32_t tphase[2] = {0u, 0u};        // the next phase of each table's barrier
+        auto load_table = [&](int wt_, int buf) {
+            const Tile tn = decode_tile(wt_, s_off, s_tiles, args.E, args.MT, BN);
+            mbar_arrive_expect_tx(&tbar[buf], (uint32_t)(tn.nrows * KBp));
+            bulk_load(tbl + (size_t)buf * BN * KBp, args.xsb + (size_t)tn.row0 * KBp, (uint32_t)(tn.nrows * KBp),
+                      &tbar[buf], pol_x);
+            tarmed |= 1u << buf;
+        };
+        if (C::BS && lane == 0 && (int)blockIdx.x < total) load_table(blockIdx.x, 0);
+        int it = 0;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
+            const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
+            const int cur = it & 1;
+            if constexpr (C::BS) {
+                ok = mbar_wait(&tbar[cur], tphase[cur], abort_flag);   // every lane reads the table
+                ok = __all_sync(0xFFFFFFFFu, ok);
+                if (!ok) break;
+                tphase[cur] ^= 1u;
+                if (lane == 0) {
+                    tarmed &= ~(1u << cur);
+                    if (w + (int)gridDim.x < total) load_table(w + gridDim.x, cur ^ 1);
+                }
+            }
+            const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
+            const int nbox = (t.nrows + C::BOX - 1) / C::BOX;
+            const uint32_t bytes = C::NUM_A * C::A_BYTES + nbox * C::BOX * 128;
+            const bool second = t.e >= args.E_split;
+            const CUtensorMap *mA = second ? &tmA2 : &tmA;
+            const int arow = (second ? t.e - args.E_split : t.e) * args.a_rows_per_expert + t.m * kBM;
+            for (int kb = 0; kb < KB; ++kb) {
+                if (lane == 0) ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) break;
+                uint8_t *sA = ring + stage * C::STAGE_BYTES;
+                uint8_t *sB = sA + C::NUM_A * C::A_BYTES;
+                if constexpr (C::BS) {
+                    // lane l holds rows l, l+32, l+64, l+96: words 4l .. 4l+3
+                    const uint8_t *tb = tbl + (size_t)cur * BN * KBp + kb;
+                    uint32_t v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = lane + 32 * i;
+                        v[i] = (n < t.nrows ? (uint32_t)tb[(size_t)n * KBp] : 127u) * 0x01010101u;
+                    }
+                    *reinterpret_cast<uint4 *>(sA + C::SFB_OFF + 16 * lane) = make_uint4(v[0], v[1], v[2], v[3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (lane == 0) {
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     armed[stage] = (int)phase;
                     tma_load_2d(sA, mA, &full[stage], kb * 128, arow, pol_w);
@@ -181,9 +256,11 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                     for (int b = 0; b < nbox; ++b)
                         tma_load_2d(sB + b * C::BOX * 128, &tmB, &full[stage], kb * 128,
                                     t.row0 + b * C::BOX, pol_x);
-                    if (++stage == NST) { stage = 0; phase ^= 1; }
                 }
+                if (++stage == NST) { stage = 0; phase ^= 1; }
             }
+        }
+        if (lane == 0) {
             if (!ok) {
                 *abort_flag = 1;
                 atomicOr(args.status, DEV_TIMEOUT);
@@ -191,6 +268,10 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
             volatile int never = 0;
             for (int s = 0; s < NST; ++s)
                 if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
+                    atomicOr(args.status, DEV_TIMEOUT);
+            // a table requested for a tile that the loop did not reach
+            for (int b = 0; b < 2; ++b)
+                if (((tarmed >> b) & 1u) && !mbar_wait(&tbar[b], tphase[b], &never))
                     atomicOr(args.status, DEV_TIMEOUT);
         }
     } else if (warp == 1 || (GATE_UP && warp == kMmaWarp2)) {
@@ -201,9 +282,14 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
             int stage = 0, pb = 0;
             uint32_t phase = 0, pphase = 0;
             bool ok = true;
+            // BS: this warp's scale columns in TMEM, weights (2^0, copied once)
+            // and the k-block's activation scales
+            const uint32_t tsfa = tmem_base + C::SF_COL + 8 * r, tsfb = tsfa + 4;
+            if constexpr (C::BS) tmem_cp_32x128b_x4(tsfa, sdesc_rows16(smem_u32(asf)));
             for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
                 const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
-                const uint32_t idesc = idesc_e4m3(kBM, (t.nrows + 15) & ~15);
+                const uint32_t idesc = C::BS ? idesc_e4m3_bs(kBM, (t.nrows + 15) & ~15)
+                                             : idesc_e4m3(kBM, (t.nrows + 15) & ~15);
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag) ||
                         !mbar_wait(&pempty[pb], pphase ^ 1, abort_flag)) { ok = false; break; }
@@ -212,8 +298,20 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                     const uint64_t da = sdesc_sw128(sa + r * C::A_BYTES);
                     const uint64_t db = sdesc_sw128(sa + C::NUM_A * C::A_BYTES);
                     const uint32_t d = tmem_base + pb * C::PCOLS + r * BN;
+                    if constexpr (C::BS) {
+                        // the scale byte of k-step k (32 elements) selected by the
+                        // descriptor and the scale addresses' top bits
+                        tmem_cp_32x128b_x4(tsfb, sdesc_rows16(sa + C::SFB_OFF));
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mma_e4m3_ss(d, da + 2 * k, db + 2 * k, idesc, k > 0);
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t sel = (uint32_t)k << 30;
+                            mma_mxf4_ss(d, da + 2 * k, db + 2 * k, idesc | idesc_sf_ids(k, k), tsfa | sel,
+                                        tsfb | sel, k > 0 ? 1u : 0u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) mma_e4m3_ss(d, da + 2 * k, db + 2 * k, idesc, k > 0);
+                    }
                     mma_commit(&empty[stage]);
                     mma_commit(&pfull[pb]);
                     if (++stage == NST) { stage = 0; phase ^= 1; }
@@ -234,19 +332,6 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
         int pb = 0;
         uint32_t pphase = 0;
         bool ok = true;
-        // activation scales of a tile's routed rows -> sx[kb][column], by
-        // asynchronous 4-byte copies (64-row tiles: the next tile's are
-        // requested as soon as every warp is done with the current ones, so
-        // that they arrive during the tile's quantisation / y stores)
-        auto stage_sx = [&](const Tile &tn) {   // warp ew: k-blocks ew, ew+8, ...; lanes: rows
-            for (int kb = ew; kb < KB; kb += kEpi8)
-                for (int c = lane; c < tn.nrows; c += 32)
-                    cp_async4(sx + kb * BN + c, args.xscale + (size_t)(tn.row0 + c) * KB + kb);
-            cp_async_commit();
-        };
-        if constexpr (!C::STAGE_SCALES) {
-            if ((int)blockIdx.x < total) stage_sx(decode_tile(blockIdx.x, s_off, s_tiles, args.E, args.MT, BN));
-        }
         for (int w = blockIdx.x; w < total; w += gridDim.x) {
             const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
             if constexpr (C::STAGE_SCALES) {
@@ -302,8 +387,6 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
             } else {
                 sg_next = __ldg(wsg);
                 if (GATE_UP) su_next = __ldg(wsu);
-                cp_async_wait<0>();                  // this thread's sx copies have landed
-                epi_sync();                          // and every thread's
             }
             for (int kb = 0; kb < KB; ++kb) {
                 const int grp = kb / C::SG, q = kb - grp * C::SG, buf = grp & 1;
@@ -336,25 +419,32 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t tb = tmem_base + ((uint32_t)(eg * 32) << 16) + pb * C::PCOLS + half * NC;
-                const float *sxk = sx + kb * BN + half * NC;   // this thread's column scales
+                const float *sxk = sx + kb * BN + half * NC;   // this thread's column scales (not BS)
                 // Load this thread's columns, hand the partial buffer back to
-                // the MMA warp, then promote the live column pairs:
-                // acc = (w_scale * x_scale) * partial + acc on fp32x2 (the
-                // roundings of the scalar form)
+                // the MMA warp, then promote the live column pairs on fp32x2:
+                // acc = (w_scale * x_scale) * partial + acc, or with BS, where
+                // the partial already carries x_scale exactly (a power of two),
+                // acc = w_scale * partial + acc -- the same single rounding
                 uint32_t pr[NC];
                 const float2 sg2 = make_float2(sg, sg), su2 = make_float2(su, su);
-                // acc[q..q+1] += (scale * x_scale[q..q+1]) * partial[q..q+1]
                 auto promote_pairs = [&](float (&acc)[NC], const float2 s2) {
 #pragma unroll
                     for (int c = 0; c < NC / 4; ++c) {
                         if (4 * c < live) {          // warp-uniform
-                            const float4 s4 = *reinterpret_cast<const float4 *>(sxk + 4 * c);
+                            float4 s4 = make_float4(1.f, 1.f, 1.f, 1.f);
+                            if constexpr (!C::BS) s4 = *reinterpret_cast<const float4 *>(sxk + 4 * c);
 #pragma unroll
                             for (int h2 = 0; h2 < 2; ++h2) {
                                 const int q = 4 * c + 2 * h2;
-                                const float2 sc = h2 == 0 ? make_float2(s4.x, s4.y) : make_float2(s4.z, s4.w);
                                 const float2 p2 = make_float2(__uint_as_float(pr[q]), __uint_as_float(pr[q + 1]));
-                                const float2 r2 = __ffma2_rn(__fmul2_rn(s2, sc), p2, make_float2(acc[q], acc[q + 1]));
+                                const float2 a2 = make_float2(acc[q], acc[q + 1]);
+                                float2 r2;
+                                if constexpr (C::BS) {
+                                    r2 = __ffma2_rn(s2, p2, a2);
+                                } else {
+                                    const float2 sc = h2 == 0 ? make_float2(s4.x, s4.y) : make_float2(s4.z, s4.w);
+                                    r2 = __ffma2_rn(__fmul2_rn(s2, sc), p2, a2);
+                                }
                                 acc[q] = r2.x;
                                 acc[q + 1] = r2.y;
                             }
@@ -389,11 +479,6 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                 }
                 if (++pb == C::NPB) { pb = 0; pphase ^= 1; }
             }
-            if constexpr (!C::STAGE_SCALES) {
-                epi_sync();                          // every warp is done with sx
-                if (w + (int)gridDim.x < total)
-                    stage_sx(decode_tile(w + gridDim.x, s_off, s_tiles, args.E, args.MT, BN));
-            }
             if (GATE_UP) {
                 // h = bf16(SiLU(g) * u) for this row (feature) and NC routed
                 // rows (SiLU with the fast division, as the bf16 epilogue)
@@ -418,7 +503,11 @@ __global__ void __launch_bounds__(Cfg8<GATE_UP, BN>::THREADS, 1)
                                           fmaxf(amax_s[2 * BN + et], amax_s[3 * BN + et]));
                     const int k = fp8_block_exp(m);
                     scale_s[et] = 1.0f / pow2f(k);   // codes are h * (1 / scale), once per column
-                    if (et < t.nrows) args.hs[(size_t)(t.row0 + et) * (args.F / 128) + t.m] = pow2f(k);
+                    if (et < t.nrows) {
+                        args.hs[(size_t)(t.row0 + et) * (args.F / 128) + t.m] = pow2f(k);
+                        if constexpr (C::BS)
+                            args.hsb[(size_t)(t.row0 + et) * ((args.F / 128 + 15) & ~15) + t.m] = (uint8_t)(k + 127);
+                    }
                 }
                 epi_sync();
                 uint8_t *hp = args.hq + (size_t)(t.row0 + half * NC) * args.F + t.m * kBM + row;
@@ -503,6 +592,7 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     g.status = (int32_t *)(ws + L.status);
     g.hq = ws + L.h;
     g.hs = (float *)(ws + L.hscale);
+    g.hsb = ws + L.hsb;
     g.y = (float *)(ws + L.y);
     g.F = F;
     g.H = H;
@@ -516,6 +606,8 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     a1.wscale = w13s;
     a1.wscale2 = sh.S > 0 ? sh.gate_up_scale : w13s;
     a1.xscale = (const float *)(ws + L.xscale);
+    a1.xsb = ws + L.xsb;
+    a1.KBp = (a1.KB + 15) & ~15;
 
     Gemm8Args a2 = g;
     a2.tiles = (const int32_t *)(ws + L.tiles_d);
@@ -526,6 +618,8 @@ cudaError_t launch_gemms_fp8(const void *w13, const float *w13s, const void *w2,
     a2.wscale = w2s;
     a2.wscale2 = sh.S > 0 ? sh.down_scale : w2s;
     a2.xscale = (const float *)(ws + L.hscale);
+    a2.xsb = ws + L.hsb;
+    a2.KBp = (a2.KB + 15) & ~15;
     if (bn == kBNFp8Decode) {
         const cudaError_t err = launch_one8<true, kBNFp8Decode>(ta, ta2, tb, a1, st);
         if (err != cudaSuccess) return err;

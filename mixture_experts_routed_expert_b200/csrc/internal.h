@@ -44,6 +44,7 @@ struct Workspace {
     size_t xscale;        // [N][H/128] f32 (e4m3 only)
     size_t h;             // [N][F] bf16 | e4m3
     size_t hscale;        // [N][F/128] f32 (e4m3 only)
+    size_t xsb, hsb;      // e4m3: the same scales as E8M0 bytes, rows of round16(H/128) / round16(F/128)
     size_t y;             // [N][H] f32 (weighted down-projection rows, by slot)
     size_t total;
 };

@@ -80,7 +80,8 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
     int bn_d, const uint4 *__restrict__ x, void *__restrict__ xperm, float *__restrict__ xscale,
     int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ tiles_g,
     int32_t *__restrict__ tiles_d, int32_t *__restrict__ perm, int32_t *__restrict__ inv,
-    int32_t *__restrict__ status, int32_t *__restrict__ zero, int nzero) {
+    int32_t *__restrict__ status, int32_t *__restrict__ zero, int nzero,
+    uint8_t *__restrict__ xsb) {
     extern __shared__ int32_t psm[];
     int32_t *cnt_all = psm;                 // [E+1] -> exclusive offsets
     int32_t *cnt_bef = cnt_all + (E + 1);   // [E] slots of e before this chunk
@@ -199,6 +200,11 @@ __global__ void __launch_bounds__(kPThreads) permute_gather_kernel(
                     if ((lane & 15) == 0) {
                         if (MODE == 2) {
                             xscale[(size_t)p * (H / 128) + v / 16] = sc;
+                            // the scale's E8M0 byte (its exponent field) in rows of
+                            // round16(H/128) bytes, for the block-scaled MMA
+                            if (xsb != nullptr)
+                                xsb[(size_t)p * ((H / 128 + 15) & ~15) + v / 16] =
+                                    (uint8_t)((__float_as_uint(sc) >> 23) & 0xFF);
                         } else {   // E8M0 byte of the power-of-two scale, rows of KBp bytes
                             const int kbp = (H / 128 + 15) & ~15;
                             reinterpret_cast<uint8_t *>(xscale)[(size_t)p * kbp + v / 16] =
@@ -307,7 +313,8 @@ cudaError_t launch_pg(const void *x, const int32_t *idx, int64_t n_slots, int K,
                     (void *)(ws + L.xperm), (float *)(ws + L.xscale), (int32_t *)(ws + L.counts),
                     (int32_t *)(ws + L.offsets), (int32_t *)(ws + L.tiles_g),
                     (int32_t *)(ws + L.tiles_d), (int32_t *)(ws + L.perm), (int32_t *)(ws + L.inv),
-                    (int32_t *)(ws + L.status), zero, nzero);
+                    (int32_t *)(ws + L.status), zero, nzero,
+                    MODE == 2 ? (uint8_t *)(ws + L.xsb) : (uint8_t *)nullptr);   // E4M3 layouts hold xsb
 }
 
 }  // namespace
