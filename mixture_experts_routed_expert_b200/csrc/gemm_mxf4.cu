@@ -79,7 +79,7 @@ struct CfgF {
     static_assert(COLS_USED <= 512, "TMEM holds 512 columns");
     static constexpr int NC = BN / 2;                   // columns per epilogue thread
     static size_t smem_bytes(int E, int KBp, int stages) {
-        return 1024 + (size_t)stages * STAGE_BYTES + 1024 + (size_t)BN * KBp +
+        return 1024 + (size_t)stages * STAGE_BYTES + 1024 + 2 * (size_t)BN * KBp +
                sizeof(float) * 5 * BN + 2 * sizeof(int) * (E + 1) + 64;
     }
 };
@@ -119,10 +119,6 @@ __device__ __forceinline__ void load_cols(uint32_t taddr, uint32_t (&r)[32], int
     tmem_ld_wait();
 }
 
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-                 : "memory");
-}
 
 template <bool GATE_UP, int BN>
 __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
@@ -138,10 +134,11 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
     uint64_t *empty = full + C::MAX_STAGES;
     uint64_t *afull = empty + C::MAX_STAGES;
     uint64_t *aempty = afull + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(aempty + 2);
+    uint64_t *tbar = aempty + 2;                                         // the two tables' barriers
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tbar + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint8_t *sxs = smem + (size_t)NST * C::STAGE_BYTES + 1024;           // [BN][KBp]
-    float *amax_s = reinterpret_cast<float *>(sxs + (size_t)BN * args.KBp);   // [4][BN]
+    uint8_t *sxs = smem + (size_t)NST * C::STAGE_BYTES + 1024;           // [2][BN][KBp]
+    float *amax_s = reinterpret_cast<float *>(sxs + 2 * (size_t)BN * args.KBp);   // [4][BN]
     float *scale_s = amax_s + 4 * BN;                                    // [BN]
     int32_t *s_off = reinterpret_cast<int32_t *>(scale_s + BN);
     int32_t *s_tiles = s_off + (args.E + 1);
@@ -156,6 +153,7 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&afull[b], 2);
             mbar_init(&aempty[b], 32 * kEpiF);
+            mbar_init(&tbar[b], 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -200,18 +198,32 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
         uint32_t phase = 0;
         for (int s = 0; s < C::MAX_STAGES; ++s) armed[s] = -1;
         bool ok = true;
-        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        // the tile's activation-scale bytes (rows n -> sxs[buf][n][0..KBp)) with
+        // one bulk copy into one of two tables, the next tile's requested as
+        // soon as the current one is ready
+        uint32_t tarmed = 0;                  // table loads issued and not yet waited for
+        uint32_t tphase[2] = {0u, 0u};        // the next phase of each table's barrier
+        auto load_table = [&](int wt_, int buf) {
+            const Tile tn = decode_tile(wt_, s_off, s_tiles, args.E, args.MT, BN);
+            mbar_arrive_expect_tx(&tbar[buf], (uint32_t)(tn.nrows * KBp));
+            bulk_load(sxs + (size_t)buf * BN * KBp, args.xsf + (size_t)tn.row0 * KBp, (uint32_t)(tn.nrows * KBp),
+                      &tbar[buf], pol_x);
+            tarmed |= 1u << buf;
+        };
+        if (do_b && lane == 0 && (int)blockIdx.x < total) load_table(blockIdx.x, 0);
+        int it = 0;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x, ++it) {
             const Tile t = decode_tile(w, s_off, s_tiles, args.E, args.MT, BN);
+            const int cur = it & 1;
             if (do_b) {
-                // the tile's activation-scale bytes, row n -> sxs[n][0..KBp)
-                const int nch = KBp / 16;
-                for (int i = lane; i < t.nrows * nch; i += 32) {
-                    const int n = i / nch, c = i - n * nch;
-                    cp_async16(sxs + n * KBp + 16 * c, args.xsf + (size_t)(t.row0 + n) * KBp + 16 * c);
+                ok = mbar_wait(&tbar[cur], tphase[cur], abort_flag);   // every lane reads the table
+                ok = __all_sync(0xFFFFFFFFu, ok);
+                if (!ok) break;
+                tphase[cur] ^= 1u;
+                if (lane == 0) {
+                    tarmed &= ~(1u << cur);
+                    if (w + (int)gridDim.x < total) load_table(w + gridDim.x, cur ^ 1);
                 }
-                cp_async_commit();
-                cp_async_wait<0>();
-                __syncwarp();
             }
             const uint64_t pol_w = s_tiles[t.e + 1] - s_tiles[t.e] > 1 ? pol_x : pol_once;
             const int arow = t.e * args.a_rows_per_expert + t.m * kBM + p * args.up_offset;
@@ -229,14 +241,20 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
                     // activation scales in the block layout: column n at word
                     // (n % 32) * 4 + n / 32 of its k-block's block, the byte
                     // repeated for the 4 slices
-                    uint32_t *sfb = reinterpret_cast<uint32_t *>(sF + C::NUM_A * C::KPB * 512);
+                    // lane l writes the words of rows l, l+32, l+64, l+96
+                    const uint8_t *tb = sxs + (size_t)cur * BN * KBp;
 #pragma unroll
-                    for (int j = 0; j < C::KPB; ++j)
-                        for (int n = lane; n < BN; n += 32) {
-                            const uint32_t b =
-                                (n < t.nrows && j < nkb) ? (uint32_t)sxs[n * KBp + kb0 + j] : 127u;
-                            sfb[j * 128 + (n & 31) * 4 + (n >> 5)] = b * 0x01010101u;
+                    for (int j = 0; j < C::KPB; ++j) {
+                        uint32_t v[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int n = lane + 32 * i;
+                            v[i] = ((n < t.nrows && j < nkb) ? (uint32_t)tb[(size_t)n * KBp + kb0 + j] : 127u) *
+                                   0x01010101u;
                         }
+                        *reinterpret_cast<uint4 *>(sF + (C::NUM_A * C::KPB + j) * 512 + 16 * lane) =
+                            make_uint4(v[0], v[1], v[2], v[3]);
+                    }
                     fence_proxy_async_smem();
                 }
                 __syncwarp();
@@ -264,6 +282,10 @@ __global__ void __launch_bounds__(CfgF<GATE_UP, BN>::THREADS, 1)
             volatile int never = 0;
             for (int s = 0; s < NST; ++s)
                 if (armed[s] >= 0 && !mbar_wait(&full[s], (uint32_t)armed[s], &never))
+                    atomicOr(args.status, DEV_TIMEOUT);
+            // a table requested for a tile that the loop did not reach
+            for (int b = 0; b < 2; ++b)
+                if (((tarmed >> b) & 1u) && !mbar_wait(&tbar[b], tphase[b], &never))
                     atomicOr(args.status, DEV_TIMEOUT);
         }
     } else if (warp == 1 || warp == C::MMA1) {
