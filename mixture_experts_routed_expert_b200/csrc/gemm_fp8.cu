@@ -4,27 +4,35 @@
 // Models", layer table: moe_w13_fp8_layer, moe_silu_mul_layer,
 // bf16_to_fp8_quantize, moe_w2_fp8_layer).
 //
-// Grouped GEMM on tcgen05 with kind::f8f6f4 (E4M3 x E4M3 -> fp32, K = 32 per
-// instruction).  Because each 128-wide k-block has its own weight and
-// activation scale, every k-block's product goes to a TMEM "partial" buffer
-// (four in rotation for gate_up, eight for down and for 16-row tiles);
-// epilogue warps read it and promote it into fp32 accumulators held in
-// registers (column pairs on fp32x2 arithmetic):
-//     acc[row, col] += (w_scale[row, kb] * x_scale[col, kb]) * partial[row, col]
-// while the MMA of the next k-block fills the other partial buffer.
+// Grouped GEMM on tcgen05, E4M3 x E4M3 -> fp32, K = 32 per instruction.
+// Because each 128-wide k-block has its own weight scale, every k-block's
+// product goes to a TMEM "partial" buffer (three in rotation for 64-row
+// gate_up tiles, three or seven for down, eight for 16-row tiles); epilogue
+// warps read it and promote it into fp32 accumulators held in registers
+// (column pairs on fp32x2 arithmetic) while later k-blocks' MMAs fill the
+// other buffers.  64/128-row tiles run kind::mxf8f6f4.block_scale with the
+// power-of-two activation scales as E8M0 block scales (the weights at 2^0),
+// so the partial already carries x_scale exactly and
+//     acc[row, col] += w_scale[row, kb] * partial[row, col]
+// (the rounding of acc += (w_scale * x_scale) * P, which 16-row tiles on
+// kind::f8f6f4 compute, from a table of the column scales).
 //   S4 (gate_up):  tile = 128 features of expert e (gate rows and up rows,
-//     two partials) x up to BN routed rows (64; 16 for a few tokens, where
-//     a tile per (expert, 128 features) is all there is to spread over the SMs).  h = bf16(SiLU(g) * u), then
-//     quantised per 128 features (the tile's 128 rows): scale = smallest power
-//     of two with max|h|/scale <= 448, codes E4M3 -> hq [N][F], hs [N][F/128].
-//   S5 (down):  tile = 128 hidden rows x up to BN routed rows;
-//     y[slot, j] = w[slot] * acc  (fp32, by original slot; combined later).
-// Warp roles: warp 0 TMA producer, warp 1 TMEM allocation + MMA issue, for
+//     two partials) x up to BN routed rows (64; 16 for a few tokens, where a
+//     tile per (expert, 128 features) is all there is to spread over the
+//     SMs).  h = bf16(SiLU(g) * u), then quantised per 128 features (the
+//     tile's 128 rows): scale = smallest power of two with max|h|/scale <=
+//     448, codes E4M3 -> hq [N][F], scales hs [N][F/128] (and their E8M0
+//     bytes for the down GEMM's block scales).
+//   S5 (down):  tile = 128 hidden rows x up to BN routed rows (64 or 128;
+//     16 for a few tokens); y[slot, j] = w[slot] * acc  (fp32, by original
+//     slot; combined later).
+// Warp roles: warp 0 TMA producer (with block scales, the whole warp also
+// writes each stage's scale block), warp 1 TMEM allocation + MMA issue, for
 // gate_up with warp 10 (warp 1 the gate MMAs, warp 10 the up MMAs of every
 // stage: one thread issuing all eight MMAs of a k-block paced the pipeline,
 // ~85 SM cycles per small tcgen05.mma against ~32 of tensor work), warps 2-9
 // promotion and epilogue (two warps per TMEM lane quarter, each owning BN/2
-// of the BN columns; promotion skips 16-column chunks past the tile's routed
+// of the BN columns; promotion skips 4-column chunks past the tile's routed
 // rows).
 #include "common.cuh"
 #include "gemm_common.cuh"
