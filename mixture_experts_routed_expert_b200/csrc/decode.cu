@@ -13,6 +13,9 @@
 // Optional shared experts (S of them, weight 1) take slots K..K+S-1 of every
 // token after its K routed slots, with their own weight tensors, and an
 // optional residual is added after the slot sum.
+// D1 is launched as a programmatic dependent of the previous kernel on the
+// stream (its blocks are placed while that kernel drains; it waits before
+// reading any input).
 // D2 is launched as a programmatic dependent of D1: before waiting for D1 it
 // prefetches its own down-projection rows into L2, so both kernels stream
 // weights from HBM at the same time.  No atomics; fixed summation order.
@@ -182,6 +185,9 @@ __global__ void __launch_bounds__(kUpWarps * 32, 1) decode_up_bf16(
     int K, int S_arg, __nv_bfloat16 *__restrict__ h) {
     __shared__ Touched tu;
     const int S = EXTRA ? S_arg : 0;   // EXTRA = false: the routed-only form
+    // Launched as a programmatic dependent of whatever precedes it on the
+    // stream: every input may come from that kernel.
+    pdl_wait();
     build_touched(idx, T, K, S, E, tu);
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = lane_id();
@@ -314,7 +320,7 @@ cudaError_t launch_decode_bf16(const void *x, const void *gate_up, const void *d
     const bool extra = S > 0 || residual != nullptr;
 #define MOE_UP(V)                                                                                 \
     launch_k(extra ? decode_up_bf16<V, true> : decode_up_bf16<V, false>, dim3(grid), blk, 0, st, \
-             false, (const uint4 *)x, (const uint4 *)gate_up, gu2, idx, T, H, F, E, K, S, h)
+             true, (const uint4 *)x, (const uint4 *)gate_up, gu2, idx, T, H, F, E, K, S, h)
     switch (vpl_up) {
         case 1: err = MOE_UP(1); break;
         case 2: err = MOE_UP(2); break;
