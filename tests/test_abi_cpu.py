@@ -54,6 +54,11 @@ def test_workspace_sizes(mod):
     assert ws(11, 1280, 896, 64, 6, decode=True) == ws(11, 1280, 896, 64, 6)   # 66 slots
     # E4M3 weights run the grouped GEMMs and need the prefill workspace
     assert ws(1, 7168, 2048, 256, 8, 1, decode=True) == ws(1, 7168, 2048, 256, 8, 1)
+    # E4M3: codes, fp32 scales and their E8M0 bytes (rows padded to 16 bytes)
+    # for x and h, and the fp32 y rows
+    N, H, F = 2048 * 8, 7168, 2048
+    need = N * (H + F + 4 * (H // 128 + F // 128) + 64 + 16 + 4 * H)
+    assert ws(2048, H, F, 256, 8, 1) >= 8192 + need
     # every workspace starts with the 8 KiB header
     assert ws(16, 256, 256, 8, 2) > mod.WORKSPACE_HEADER_BYTES == 8192
     assert ws(16, 100, 896, 64, 6) == 0          # H % 128 != 0
