@@ -143,18 +143,21 @@ MOE_API moe_status_t moe_experts_prefill(const void *hidden_states, const void *
                                  size_t workspace_bytes, void *stream);
 
 /*
- * Routed-experts forward, decode form: a fused gather-GEMV for a few tokens
- * (model card op "deepseek_ocr2_moe_experts_decode", n_tokens about 1-4).
- * Same arguments, layouts and results as moe_experts_prefill, workspace from
- * moe_experts_workspace_size(..., 1).  Tuned for T * K <= 64.  bf16 weights
- * with T <= 16 and H, F <= 2048: one kernel launch (expert dedup, gate/up
- * GEMV with SiLU*up, down GEMV, router-weight scale and the fixed-order
- * top-K combine), launched as a programmatic dependent of the previous
- * kernel on the stream (it reads no input before that kernel has finished);
- * it counts on the workspace header being zero (see the conventions above).
- * E4M3 and MXFP4 weights: the grouped GEMMs with 16-row activation tiles.
- * Larger calls are served by the prefill kernels (same results within the
- * parity tolerance).
+ * Routed-experts forward, decode form for a few tokens (model card op
+ * "deepseek_ocr2_moe_experts_decode", n_tokens about 1-4).  Same arguments,
+ * layouts and results as moe_experts_prefill, workspace from
+ * moe_experts_workspace_size(..., 1).
+ *  - bf16 weights, T * K <= 16, H, F <= 2048: a fused gather-GEMV pair.
+ *    The first kernel streams the gate and up rows of every touched expert
+ *    once and writes h = bf16(SiLU(g) * u) for the slots routed to it; the
+ *    second, a programmatic dependent of the first, streams the touched down
+ *    rows once per hidden row, scales by the router weights and sums each
+ *    token's K slots in k order.  The first kernel is itself launched as a
+ *    programmatic dependent of the previous kernel on the stream and reads
+ *    no input before that kernel has finished.
+ *  - E4M3 and MXFP4 weights, and larger bf16 calls: the prefill kernels
+ *    (E4M3 / MXFP4 with 16-row activation tiles at these sizes); same
+ *    results within the parity tolerance.
  */
 MOE_API moe_status_t moe_experts_decode(const void *hidden_states, const void *gate_up_proj,
                                 const void *down_proj, const int32_t *top_k_index,
