@@ -44,7 +44,8 @@ def build(force=False, verbose=False):
                 raise RuntimeError("nvcc failed on %s" % s)
     if force or jobs or _stale(LIB, objs):
         tmp = LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call([NVCC, "-shared", "-o", tmp, *objs, "-Xcompiler", "-fPIC"])
+        subprocess.check_call([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp,
+                               *objs, "-Xcompiler", "-fPIC"])
         os.replace(tmp, LIB)
     return LIB
 
